@@ -1,0 +1,100 @@
+"""Plant plausible mistakes in copies of the CPU oracle and check that each one
+fails at least one pin (so the pins do constrain every step of the oracle).
+
+The mistakes are planted in the C source of a temporary copy, on the CPU; the
+real oracle is never modified.  Each mutant runs in a child process, since a
+broken copy may also crash (which counts as caught).
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+import oracle
+
+_WRITE = "    /* gated delta write on the W selected slots (item 3) */\n"
+_READ = "    /* sparse read after the write (item 4) */\n"
+_READ_END = "    if (io->o)\n"
+
+
+def _swap_read_write(src):
+    i, j, k = src.index(_WRITE), src.index(_READ), src.index(_READ_END)
+    return src[:i] + src[j:k] + src[i:j] + src[k:]
+
+
+MUTANTS = {
+    "second-half-uses-first-half": lambda s: s.replace(
+        "b += (double)x[dh + c] * (double)C2[", "b += (double)x[c] * (double)C2["),
+    "halves-meet-swapped-codebooks": lambda s: s.replace(
+        "a += (double)x[c] * (double)C1[", "a += (double)x[c] * (double)C2[").replace(
+        "b += (double)x[dh + c] * (double)C2[", "b += (double)x[dh + c] * (double)C1["),
+    "slot-numbering-transposed": lambda s: s.replace(
+        "c->slot = (int64_t)w->h1[a].id * n + w->h2[b].id;",
+        "c->slot = (int64_t)w->h2[b].id * n + w->h1[a].id;"),
+    "slot-tie-break-reversed": lambda s: s.replace(
+        "return (a->slot < b->slot) ? -1 : (a->slot > b->slot);",
+        "return (a->slot > b->slot) ? -1 : (a->slot < b->slot);"),
+    "half-tie-break-reversed": lambda s: s.replace(
+        "return (a->id < b->id) ? -1 : (a->id > b->id);",
+        "return (a->id > b->id) ? -1 : (a->id < b->id);"),
+    "half-topk-keeps-smallest": lambda s: s.replace(
+        "  if (a->s > b->s) return -1;\n  if (a->s < b->s) return 1;\n  return (a->id",
+        "  if (a->s < b->s) return -1;\n  if (a->s > b->s) return 1;\n  return (a->id", 1),
+    "candidate-grid-short-by-one": lambda s: s.replace(
+        "for (int b = 0; b < k; ++b) {", "for (int b = 0; b + 1 < k; ++b) {"),
+    "forget-gate-dropped": lambda s: s.replace(
+        "const double mt = a * (double)row[col];", "const double mt = (double)row[col];"),
+    "forget-gate-on-new-value": lambda s: s.replace(
+        "row[col] = (float)((1.0 - c) * mt + c * (double)vt[col]);",
+        "row[col] = (float)(a * ((1.0 - c) * (double)row[col] + c * (double)vt[col]));"),
+    "delta-sign-flipped": lambda s: s.replace(
+        "row[col] = (float)((1.0 - c) * mt + c * (double)vt[col]);",
+        "row[col] = (float)((1.0 + c) * mt - c * (double)vt[col]);"),
+    "beta-dropped": lambda s: s.replace(
+        "const double c = be * ww[j];", "const double c = ww[j];"),
+    "uniform-weights": lambda s: s.replace(
+        "wt_out[j] = exp((double)w->cand[j].s - m) / z;", "wt_out[j] = 1.0 / n_sel;"),
+    "softmax-of-negated-scores": lambda s: s.replace(
+        "wt_out[j] = exp((double)w->cand[j].s - m) / z;",
+        "wt_out[j] = exp(m - (double)w->cand[j].s) / z;"),
+    "read-before-write": _swap_read_write,
+    "read-uses-write-weights": lambda s: s.replace(
+        "acc[col] += rw[j] * (double)row[col];", "acc[col] += ww[j % d->W] * (double)row[col];"),
+    "fp64-candidate-order": lambda s: s.replace(
+        "float s = w->h1[a].s + w->h2[b].s;          /* float32 sum */",
+        "float s = (float)(w->s64_1[w->h1[a].id] + w->s64_2[w->h2[b].id]);"),
+}
+
+
+@pytest.fixture(scope="module")
+def mutant_dir():
+    with tempfile.TemporaryDirectory(prefix="sdm_oracle_mut_") as d:
+        yield d
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, mutant_dir):
+    with open(oracle.ORACLE_SRC) as f:
+        src = f.read()
+    bad = MUTANTS[name](src)
+    assert bad != src, "mutation %s did not apply" % name
+    c = os.path.join(mutant_dir, name + ".c")
+    so = os.path.join(mutant_dir, name + ".so")
+    with open(c, "w") as f:
+        f.write(bad)
+    oracle.compile_source(c, so)
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import pins\n"
+            "bad = []\n"
+            "for pin in pins.ALL_PINS:\n"
+            "    try:\n"
+            "        pin(%r)\n"
+            "    except AssertionError:\n"
+            "        bad.append(pin.__name__)\n"
+            "print(bad)\n"
+            "sys.exit(1 if bad else 0)\n") % (here, os.path.dirname(here), so)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, "no pin catches the mutation %r" % name
