@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of the SDM forward pass: token-heads/s at N = 2^20 slots per head.
+
+Workload (default): the pages-scale workload -- B=2, H=4, T=8192, d_qk=128
+(halves of 64), codebooks 1024 x 64 per head (N = 2^20), d_v=64, k=64, W=R=64,
+bf16 inputs, float32 state.  One step = one full forward pass (scoring,
+selection, gated delta recurrence, reads) over the batch.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdm|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own shard of
+the batch (weak scaling, no collective on the data path); time is the max over
+ranks of the summed per-step CUDA-event times, with L2 flushed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SDM forward token-heads/s at N=2^20; slot-traffic HBM GB/s vs B200 peak"
+UNIT = "token-heads/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["sdm", "reference"], default="sdm")
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def workload_desc(cfg):
+    return ("%s: B=%d H=%d T=%d d_qk=%d d_v=%d n_sub=%d (N=%d) k=%d W=%d R=%d %s inputs, f32 state"
+            % (cfg.name, cfg.B, cfg.H, cfg.T, cfg.d_qk, cfg.d_v, cfg.n_sub, cfg.N, cfg.k, cfg.W,
+               cfg.R, cfg.in_dtype))
+
+
+# ----------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.proc = None
+        self.path = None
+        self.uuid = uuid
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="sdm_clocks_", suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- cpu baseline
+def cpu_baseline(cfg, target_s: float, b0: int = 0):
+    """The oracle, as it stands, on a bounded sample of the workload: the first
+    min(B*H, host threads) heads over a prefix of T_s steps."""
+    import numpy as np
+    import oracle
+    from synth import gen_inputs
+
+    nthr = host_threads()
+    nheads = min(cfg.BH, nthr)
+    sub = cfg.with_(B=1, H=1)
+    # calibrate on one head
+    one = gen_inputs(sub, t_end=16, b0=b0)
+    npi = {k: v.numpy() for k, v in one.items()}
+    d = dict(cfg.dims(), B=1, H=1, T=16)
+    t = time.perf_counter()
+    oracle.forward(npi, d)
+    per_step = (time.perf_counter() - t) / 16
+    waves = (nheads + nthr - 1) // nthr
+    T_s = int(max(16, min(cfg.T, target_s / max(per_step * waves, 1e-9))))
+    heads = [(hh // cfg.H, hh % cfg.H) for hh in range(nheads)]
+    Bs = cfg.with_(B=max(b for b, _ in heads) + 1)
+    inp = gen_inputs(Bs, t_end=T_s, b0=b0)
+    npi = {k: v.numpy() for k, v in inp.items()}
+    dd = dict(Bs.dims(), T=T_s)
+    flat = [b * cfg.H + h for b, h in heads]
+    t = time.perf_counter()
+    oracle.forward(npi, dd, heads=flat, nthreads=nthr)
+    el = time.perf_counter() - t
+    return {"value": nheads * T_s / el, "unit": UNIT, "cores": min(nthr, nheads), "kind": "oracle",
+            "sample": "%d heads x first %d steps of %s (oracle C, float64, %d threads, %.1f s)"
+                      % (nheads, T_s, cfg.name, min(nthr, nheads), el)}
+
+
+# ---------------------------------------------------------------------- sdm arm
+def run_sdm(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_memory_linear_scoring_b200 as sdm
+    from synth import gen_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dims = sdm.make_dims(**cfg.dims())
+    plan = sdm.query_plan(dims)
+    inp = gen_inputs(cfg, b0=rank * cfg.B)
+    dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
+    d = {n: inp[n].to(dev, dt).contiguous() for n in ("q", "k", "v", "C1", "C2")}
+    for n in ("alpha", "beta"):
+        d[n] = inp[n].to(dev).contiguous()
+    M = inp["M0"].to(dev).contiguous()
+    del inp
+    o = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nph = 4 * plan["chunks"]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(nph)]
+
+    def step(events=None):
+        sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], M,
+                    topk=cfg.k, W=cfg.W, R=cfg.R, o=o, events=events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, info = sdm.device_status()
+    if st != 0:
+        raise RuntimeError("device status %d (info %d) after warm-up" % (st, info))
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    clocks = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    total = 0.0
+    phase = [0.0, 0.0, 0.0]
+    for _ in range(args.steps):
+        flush.zero_()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record()
+        step(ev)
+        s1.record()
+        s1.synchronize()
+        total += s0.elapsed_time(s1)
+        for c in range(plan["chunks"]):
+            for j in range(3):
+                phase[j] += ev[4 * c + j].elapsed_time(ev[4 * c + j + 1])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    st, info = sdm.device_status()
+    if st != 0:
+        raise RuntimeError("device status %d (info %d) after timing" % (st, info))
+    t_max = total
+    if world > 1:
+        tt = torch.tensor([total] + phase, dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt[0])
+        phase = [float(x) for x in tt[1:]]
+
+    # ---- end to end through the public API: pinned host inputs -> device ->
+    # forward -> o back to pinned host memory, every step
+    e2e = None
+    if not args.no_e2e:
+        names = ("q", "k", "v", "alpha", "beta")
+        host = {n: torch.empty_like(d[n], device="cpu").pin_memory() for n in names}
+        for n in names:
+            host[n].copy_(d[n])
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        dbuf = {n: torch.empty_like(d[n]) for n in names}
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+        d2h = o_host.numel() * o_host.element_size()
+
+        def e2e_step():
+            for n in names:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            sdm.forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], d["C1"],
+                        d["C2"], M, topk=cfg.k, W=cfg.W, R=cfg.R, o=o)
+            o_host.copy_(o, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        et = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record()
+            e2e_step()
+            s1.record()
+            s1.synchronize()
+            et += s0.elapsed_time(s1)
+        if world > 1:
+            tt = torch.tensor([et], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            et = float(tt[0])
+        e2e = {"value": world * cfg.BH * cfg.T * args.steps / (et / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        return None
+    pk, src = peaks()
+    K = args.steps
+    th = cfg.BH * cfg.T
+    value = world * th * K / (t_max / 1e3)
+    names = ["score", "merge_plan", "recur"]
+    shares = {n: phase[i] / max(1e-12, sum(phase)) for i, n in enumerate(names)}
+    per = {n: phase[i] / K for i, n in enumerate(names)}
+    dom = max(names, key=lambda n: per[n])
+    slot_bytes = th * (2 * cfg.W + cfg.R) * cfg.d_v * 4
+    score_flops = th * 4 * cfg.n_sub * cfg.d_qk
+    if dom == "recur":
+        roof = {"kernel": "k_recur", "bound": "hbm",
+                "achieved": slot_bytes / (per["recur"] / 1e3) / 1e9,
+                "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    elif dom == "score" and plan["tensor_core_scoring"]:
+        roof = {"kernel": "k_score_tc", "bound": "tensor",
+                "achieved": score_flops / (per["score"] / 1e3) / 1e12,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        # CUDA-core kernels: float32 FMA peak = 148 SMs x 128 lanes x 2 x max clock
+        fp32_peak = 148 * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        kname = "k_score_simt" if dom == "score" else "k_merge_plan"
+        roof = {"kernel": kname, "bound": "alu",
+                "achieved": (score_flops / (per[dom] / 1e3) / 1e12) if dom == "score" else None,
+                "peak": fp32_peak, "unit": "TFLOP/s"}
+    roof["frac"] = (roof["achieved"] / roof["peak"]) if roof["achieved"] else None
+    roof["traffic"] = None
+    roof["peak_source"] = src
+    rec_gbs = slot_bytes / (per["recur"] / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": t_max / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world,
+                   "heads": cfg.H, "seq_len": cfg.T, "parallelism": "dp%d (heads sharded, no collective)" % world,
+                   "l2": "flushed between steps (256 MiB write)"},
+        "roofline": roof,
+        "slot_traffic": {"bytes_per_step": slot_bytes, "recur_gbs": rec_gbs,
+                         "recur_frac_of_8TBs": rec_gbs / 8000.0,
+                         "recur_frac_of_measured": rec_gbs / pk["hbm_gbs"],
+                         "whole_step_gbs": slot_bytes / (t_max / K / 1e3) / 1e9},
+        "phases_ms": per, "phase_share": shares, "plan": plan,
+        "gpu_launches": int(plan["launches_per_call"] * K),
+        "clocks": clk, "e2e": e2e,
+    }
+    return out
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, cfg):
+    """The oracle on the host cores, each step a bounded sample of the workload."""
+    import oracle
+    from synth import gen_inputs
+
+    budget = 150.0 / max(1, args.steps + args.warmup)   # seconds per step
+    nthr = host_threads()
+    nheads = min(cfg.BH, nthr)
+    sub = cfg.with_(B=1, H=1)
+    one = gen_inputs(sub, t_end=16)
+    npi = {k: v.numpy() for k, v in one.items()}
+    t = time.perf_counter()
+    oracle.forward(npi, dict(cfg.dims(), B=1, H=1, T=16))
+    per_step = (time.perf_counter() - t) / 16
+    T_s = int(max(8, min(cfg.T, budget / max(per_step, 1e-9))))
+    heads = list(range(nheads))
+    Bs = cfg.with_(B=(nheads - 1) // cfg.H + 1)
+    inp = gen_inputs(Bs, t_end=T_s)
+    npi = {k: v.numpy() for k, v in inp.items()}
+    dd = dict(Bs.dims(), T=T_s)
+    for _ in range(args.warmup):
+        oracle.forward(npi, dd, heads=heads, nthreads=nthr)
+    tot = 0.0
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle.forward(npi, dd, heads=heads, nthreads=nthr)
+        tot += time.perf_counter() - t
+    th = nheads * T_s * args.steps
+    value = th / tot
+    sample = "%d heads x first %d steps of %s per step (oracle C, float64, %d threads)" % (
+        nheads, T_s, cfg.name, min(nthr, nheads))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(cfg), "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(nthr, nheads),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    from synth import config
+    cfg = config(args.config)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    out = run_sdm(args, cfg, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

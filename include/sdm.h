@@ -1,0 +1,180 @@
+/*
+ * sdm.h -- C ABI of the Sparse Delta Memory (SDM) forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The operation (SDM technical summaries of arXiv 2607.07386, gist.science,
+ * es "Resumen Tecnico: Memoria Delta Dispersa (SDM)" / fr "Resume Technique :
+ * Memoire Delta Creuse (SDM)", section "Mecanismo Central" items 1-4): each
+ * (b,h) head keeps a slot table M in R^{N x d_v}, N = n_sub^2.  At step t the
+ * projected key k'_t and query q'_t are each cut into two contiguous halves;
+ * half 1 is scored against codebook C1, half 2 against C2 (n_sub rows of
+ * d_qk/2 each); each half keeps its top-k; the k x k outer-sum candidates give
+ * slot i = i1 * n_sub + i2 with score s1[i1] + s2[i2] (float32); k' selects the
+ * top-W write slots, q' the top-R read slots (lower index wins ties).  Each
+ * write slot is gated then delta-updated,
+ *     M~[i] = alpha_t * M[i];  M[i] = M~[i] + beta_t * w_i * (v_t - M~[i]),
+ * with w = softmax over the W selected write scores; other slots are left
+ * bit-identical.  o_t = sum_r u_r * M_t[r] over the R read slots, u = softmax
+ * over the R read scores, taken after step t's write.
+ *
+ * Conventions for every entry point:
+ *  - Pointers are CUDA device pointers unless stated otherwise; the caller
+ *    allocates and owns every buffer, including the workspace.  The library
+ *    allocates no device memory and keeps no state between calls.
+ *  - Layouts are dense row-major, no padding:
+ *      q, k   [B][H][T][d_qk]   (in_dtype)
+ *      v      [B][H][T][d_v]    (in_dtype)
+ *      alpha, beta [B][H][T]    float32
+ *      C1, C2 [H][n_sub][d_qk/2] (in_dtype)
+ *      M      [B][H][N][d_v]    float32, N = n_sub^2
+ *      o      [B][H][T][d_v]    float32
+ *      idx_w / w_w [B][H][T][W] int32 / float32 (idx_r / w_r likewise with R)
+ *  - Every device pointer must be 16-byte aligned; outputs must not alias
+ *    inputs or each other.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work
+ *    is enqueued on it and the call returns without waiting; results are
+ *    valid after the stream is synchronised.
+ *  - Return value: SDM_OK, or an sdm_status code.  Argument errors are found
+ *    on the host before anything is enqueued.  A failure to enqueue returns
+ *    SDM_ERR_CUDA.  A check made by the kernels themselves (an index out of
+ *    range, a bounded wait that ran out) is recorded in the workspace's status
+ *    word; read it with sdm_get_device_status after synchronising.
+ *  - No C++ exception crosses this boundary.
+ */
+#ifndef SDM_H_
+#define SDM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SDM_API __attribute__((visibility("default")))
+#else
+#define SDM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem sizes.  in_dtype applies to q', k', v, C1 and C2. */
+typedef struct sdm_dims {
+  int32_t B;        /* batch */
+  int32_t H;        /* heads */
+  int32_t T;        /* steps */
+  int32_t d_qk;     /* projected key/query width (even); halves of d_qk/2 */
+  int32_t d_v;      /* slot row width: 4, 8, 16, 32, 64 or 128 */
+  int32_t n_sub;    /* rows per sub-key codebook; N = n_sub^2 < 2^31 */
+  int32_t k;        /* per-half top-k, 1 <= k <= n_sub */
+  int32_t W;        /* write slots per step, 1 <= W <= k^2 */
+  int32_t R;        /* read slots per step, 1 <= R <= k^2 */
+  int32_t in_dtype; /* SDM_DTYPE_F32 or SDM_DTYPE_BF16 */
+} sdm_dims;
+
+enum { SDM_DTYPE_F32 = 0, SDM_DTYPE_BF16 = 1 };
+
+enum {
+  SDM_OK = 0,
+  SDM_ERR_NULL = 1,        /* a required pointer is NULL */
+  SDM_ERR_DIMS = 2,        /* sizes out of range or inconsistent */
+  SDM_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  SDM_ERR_WORKSPACE = 4,   /* workspace missing or smaller than sdm_workspace_bytes */
+  SDM_ERR_UNSUPPORTED = 5, /* valid sizes this build has no kernel for */
+  SDM_ERR_CUDA = 6,        /* a CUDA call failed while enqueueing */
+  SDM_ERR_DEVICE = 7       /* a kernel's own check fired (see sdm_get_device_status) */
+};
+
+/* Device status bits recorded by the kernels (sdm_get_device_status). */
+enum {
+  SDM_DEV_BAD_INDEX = 1,    /* a slot or list index outside its range (access skipped) */
+  SDM_DEV_CAPACITY = 2,     /* a per-row survivor list overflowed its capacity */
+  SDM_DEV_TIMEOUT = 4,      /* a bounded wait ran out (work skipped) */
+  SDM_DEV_BAD_LIST = 8      /* a given selection list repeats a slot within one step (applied in order) */
+};
+
+/*
+ * Bytes of device workspace sdm_forward / sdm_select / sdm_recur need for
+ * `dims` (0 if dims are invalid).  Depends on dims only.  The workspace
+ * holds per-call scratch (per-half survivor lists, the write/read plans of
+ * the recurrence, a status word); its contents need not be initialised and
+ * are overwritten by each call.
+ */
+SDM_API size_t sdm_workspace_bytes(const sdm_dims* dims);
+
+/*
+ * Full forward pass ("Mecanismo Central" items 1-4).
+ *   q, k, v, alpha, beta, C1, C2: inputs (read only), layouts above.
+ *   M_inout: read as M_0 and overwritten with M_T.
+ *   o_out:   written with o_0 .. o_{T-1}.
+ *   workspace: ws_bytes >= sdm_workspace_bytes(dims) device bytes.
+ * Calls on the same workspace must be serialised (same stream or an event).
+ */
+SDM_API int sdm_forward(const void* q, const void* k, const void* v, const float* alpha,
+                const float* beta, const void* C1, const void* C2, float* M_inout,
+                float* o_out, const sdm_dims* dims, void* workspace, size_t ws_bytes,
+                void* stream);
+
+/*
+ * Selection only (item 2): the write list from k' and the read list from q',
+ * each in rank order (score descending, slot ascending), with their softmax
+ * weights.  idx_w / w_w: [B][H][T][W]; idx_r / w_r: [B][H][T][R].
+ * v, alpha, beta, M are not needed.
+ */
+SDM_API int sdm_select(const void* q, const void* k, const void* C1, const void* C2, int32_t* idx_w,
+               float* w_w, int32_t* idx_r, float* w_r, const sdm_dims* dims, void* workspace,
+               size_t ws_bytes, void* stream);
+
+/*
+ * Recurrence only (items 3-4) from given selection lists: the write slots
+ * idx_w with weights w_w and the read slots idx_r with weights u = w_r, as
+ * sdm_select produces them (any order within a step).  The W slots of one
+ * step should be distinct, as should the R slots: a repeat is applied in list
+ * order and flagged (SDM_DEV_BAD_LIST); a slot outside [0, N) is skipped and
+ * flagged (SDM_DEV_BAD_INDEX).  q, k, C1, C2 are not needed; in_dtype applies
+ * to v; d_qk and n_sub still give N and must be valid.
+ */
+SDM_API int sdm_recur(const void* v, const float* alpha, const float* beta, const int32_t* idx_w,
+              const float* w_w, const int32_t* idx_r, const float* w_r, float* M_inout,
+              float* o_out, const sdm_dims* dims, void* workspace, size_t ws_bytes,
+              void* stream);
+
+/*
+ * sdm_forward that also records caller-created CUDA events (cudaEvent_t) on
+ * `stream` at the boundaries of its kernel phases, for timing: for time chunk c
+ * (see sdm_query_plan) events[4c+0] before scoring, [4c+1] after scoring,
+ * [4c+2] after the merge/plan kernel, [4c+3] after the recurrence kernel.
+ * Boundaries past n_events are not recorded.  Same results as sdm_forward.
+ */
+SDM_API int sdm_forward_timed(const void* q, const void* k, const void* v, const float* alpha,
+                              const float* beta, const void* C1, const void* C2, float* M_inout,
+                              float* o_out, const sdm_dims* dims, void* workspace,
+                              size_t ws_bytes, void* stream, void* const* events, int n_events);
+
+/*
+ * How the library will run `dims` (host only, no GPU work).  Writes up to n
+ * values into out: [0] tensor-core scoring (1) or CUDA-core scoring (0),
+ * [1] survivor capacity per half-row, [2] steps per plan block P,
+ * [3] slot parts per head G, [4] steps per time chunk, [5] number of chunks,
+ * [6] kernel launches per sdm_forward call.  Returns SDM_OK or a dims error.
+ */
+SDM_API int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n);
+
+/*
+ * Copy the device status word of the last call made with `workspace` into
+ * *status (SDM_DEV_* bits, 0 = clean) and *info (the first offending index, or
+ * -1).  Synchronises `stream`.  Returns SDM_OK, SDM_ERR_NULL,
+ * SDM_ERR_WORKSPACE or SDM_ERR_CUDA.
+ */
+SDM_API int sdm_get_device_status(const void* workspace, size_t ws_bytes, int32_t* status,
+                          int32_t* info, void* stream);
+
+/* Static text for a return code (never NULL). */
+SDM_API const char* sdm_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+SDM_API int sdm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDM_H_ */

@@ -1,0 +1,396 @@
+// merge_plan.cu -- product-key merge, softmax weights, and the recurrence plan.
+//
+// SDM summaries (gist.science 2607.07386), "Mecanismo Central" item 2: the top-W
+// write slots (from k') and top-R read slots (from q') are the best of the k x k
+// outer-sum candidates of the two halves' top-k lists,
+//   topk(s1 (+) s2) = topk(topk(s1) (+) topk(s2)),   slot = i1 * n + i2,
+// ordered by (float32 sum descending, slot ascending).  Item 3 weights: w =
+// softmax over the W selected write scores, u = softmax over the R read scores.
+//
+// Merge (one warp per (step, side)): sort each half's survivors, evaluate the
+// "staircase" candidates (a, b) with (a+1)(b+1) <= n_sel (a, b = ranks in the
+// two halves), sort them, and take the first n_sel.  This is exact when every
+// candidate outside the staircase scores strictly below the n_sel-th: the
+// largest outside score is attained on the staircase's frontier (row a, column
+// bmax(a)), since sums fall along each row; if the frontier check fails, an
+// exact search over all k x k candidates runs instead.
+//
+// Plan (one CTA per (head, block of P steps)): the block's W+R entries per step
+// are grouped for the recurrence kernel.  Each slot belongs to one of G parts
+// (a hash of the slot); records are laid out part by part: first the slots
+// used once in the block, then the slots used several times, grouped by slot
+// in time order (write before read within a step).  A record is
+//   int4 {slot, (step_in_block << 1) | is_read, weight bits, chain length},
+// chain length = number of records of that slot in the block on its first
+// record, 0 on the others.
+#include "sdm_internal.cuh"
+
+namespace sdm {
+
+constexpr uint32_t kEmpty = 0xffffffffu;
+constexpr uint32_t kInvalid = 0xffffffffu;
+
+struct MergeLayout {
+  size_t ent_slot, ent_w, stair, misc, uni, total;
+  int Sk, Sc, HS, warps;
+  size_t per_warp, phase2;
+};
+
+__host__ __device__ inline int p2(int x) {
+  int p = 2;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+__host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
+
+__host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
+  MergeLayout L;
+  L.Sk = p2(p.C);
+  L.Sc = p2(p.ncW > p.ncR ? p.ncW : p.ncR);
+  L.HS = p2(2 * p.E);
+  L.warps = warps;
+  size_t o = 0;
+  L.ent_slot = o; o = al16(o + size_t(p.E) * 4);
+  L.ent_w = o; o = al16(o + size_t(p.E) * 4);
+  L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR) * 4);
+  L.misc = o; o = al16(o + size_t(5 * (kMaxParts + 1) + 8) * 4);
+  L.uni = o;
+  L.per_warp = size_t(2 * L.Sk + L.Sc) * 8;
+  L.phase2 = al16(size_t(L.HS) * 4) + al16(size_t(L.HS)) + al16(size_t(p2(p.E)) * 2);
+  const size_t ph1 = L.per_warp * warps;
+  o += (ph1 > L.phase2 ? ph1 : L.phase2);
+  L.total = al16(o);
+  return L;
+}
+
+size_t merge_smem_bytes(const Plan& p, int warps) { return merge_layout(p, warps).total; }
+
+// ------------------------------------------------------------------ merge (warp)
+// Exact top-n_sel of all k*k candidates by a bitwise search over the 64-bit
+// keys, counting by enumeration.  Used only when the staircase is not provably
+// sufficient.  Leaves the n_sel best keys, descending, in cand[0..n_sel).
+__device__ void merge_full(const uint64_t* h1, const uint64_t* h2, int k, int n, int n_sel,
+                           uint64_t* cand) {
+  const int lane = threadIdx.x & 31;
+  const int kk = k * k;
+  uint64_t prefix = 0;
+  for (int bit = 63; bit >= 0; --bit) {
+    const uint64_t probe = prefix | (uint64_t(1) << bit);
+    int cnt = 0;
+    for (int i = lane; i < kk; i += 32) {
+      const int a = i / k, b = i - a * k;
+      const float v = key_val(h1[a]) + key_val(h2[b]);
+      const uint32_t slot = key_idx(h1[a]) * uint32_t(n) + key_idx(h2[b]);
+      cnt += make_key(v, slot) >= probe;
+    }
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= n_sel) prefix = probe;
+  }
+  // prefix is the n_sel-th largest key; gather the keys >= prefix (exactly n_sel)
+  int base = 0;
+  for (int i0 = 0; i0 < kk; i0 += 32) {
+    const int i = i0 + lane;
+    uint64_t key = 0;
+    bool take = false;
+    if (i < kk) {
+      const int a = i / k, b = i - a * k;
+      const float v = key_val(h1[a]) + key_val(h2[b]);
+      const uint32_t slot = key_idx(h1[a]) * uint32_t(n) + key_idx(h2[b]);
+      key = make_key(v, slot);
+      take = key >= prefix;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (take) cand[base + __popc(m & ((1u << lane) - 1u))] = key;
+    base += __popc(m);
+  }
+  __syncwarp();
+  const int S = p2(n_sel);
+  for (int i = n_sel + lane; i < S; i += 32) cand[i] = 0;
+  __syncwarp();
+  warp_sort_desc(cand, S);
+}
+
+// Sorted top-k of one half's survivors into h[0..k); returns false when the
+// survivor count is out of range.
+__device__ bool half_topk(const uint2* sv, int cnt, int k, int C, uint64_t* h) {
+  const int lane = threadIdx.x & 31;
+  if (cnt < k || cnt > C) return false;
+  const int S = p2(cnt);
+  for (int i = lane; i < S; i += 32)
+    h[i] = (i < cnt) ? make_key(__uint_as_float(sv[i].x), sv[i].y) : uint64_t(0);
+  __syncwarp();
+  warp_sort_desc(h, S);
+  return true;
+}
+
+__device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
+                          int n_sel, const uint32_t* stair, int nc, const uint32_t* front, int nf,
+                          uint64_t* h1, uint64_t* h2, uint64_t* cand, float* w_out,
+                          uint32_t* slot_out, DevStatus* st, int info) {
+  const int lane = threadIdx.x & 31;
+  const bool ok1 = half_topk(sv1, c1, p.k, p.C, h1);
+  const bool ok2 = half_topk(sv2, c2, p.k, p.C, h2);
+  if (!ok1 || !ok2) {
+    if (lane == 0) dev_flag(st, SDM_DEV_CAPACITY, info);
+    for (int i = lane; i < n_sel; i += 32) { w_out[i] = 0.f; slot_out[i] = kInvalid; }
+    __syncwarp();
+    return;
+  }
+  const uint32_t n = uint32_t(p.n);
+  const int Sc = p2(nc);
+  for (int i = lane; i < Sc; i += 32) {
+    uint64_t key = 0;
+    if (i < nc) {
+      const uint32_t ab = stair[i];
+      const int a = ab & 0xffff, b = ab >> 16;
+      const float v = key_val(h1[a]) + key_val(h2[b]);
+      key = make_key(v, key_idx(h1[a]) * n + key_idx(h2[b]));
+    }
+    cand[i] = key;
+  }
+  __syncwarp();
+  warp_sort_desc(cand, Sc);
+  // frontier check: every candidate outside the staircase must score strictly
+  // below the n_sel-th staircase candidate
+  const uint32_t tau = uint32_t(cand[n_sel - 1] >> 32);
+  bool bad = false;
+  for (int i = lane; i < nf; i += 32) {
+    const uint32_t ab = front[i];
+    const int a = ab & 0xffff, b = ab >> 16;
+    bad |= f2ord(key_val(h1[a]) + key_val(h2[b])) >= tau;
+  }
+  if (__any_sync(0xffffffffu, bad)) merge_full(h1, h2, p.k, p.n, n_sel, cand);
+  // softmax over the selected float32 scores
+  const float m = key_val(cand[0]);
+  float zs = 0.f;
+  for (int i = lane; i < n_sel; i += 32) zs += expf(key_val(cand[i]) - m);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
+  const float inv = 1.f / zs;
+  for (int i = lane; i < n_sel; i += 32) {
+    w_out[i] = expf(key_val(cand[i]) - m) * inv;
+    slot_out[i] = key_idx(cand[i]);
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------------ kernel
+__global__ void __launch_bounds__(kMergeThreads)
+k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const MergeLayout L = merge_layout(p, p.merge_warps);
+  uint32_t* ent_slot = reinterpret_cast<uint32_t*>(smem + L.ent_slot);
+  float* ent_w = reinterpret_cast<float*>(smem + L.ent_w);
+  uint32_t* stairW = reinterpret_cast<uint32_t*>(smem + L.stair);
+  uint32_t* frontW = stairW + p.ncW;
+  uint32_t* stairR = frontW + p.nfW;
+  uint32_t* frontR = stairR + p.ncR;
+  int* cnt_s = reinterpret_cast<int*>(smem + L.misc);
+  int* cnt_m = cnt_s + (kMaxParts + 1);
+  int* base = cnt_m + (kMaxParts + 1);
+  int* mbase = base + (kMaxParts + 1);
+  int* fill = mbase + (kMaxParts + 1);
+  int* misc = fill + (kMaxParts + 1);  // [0] n_multi
+  unsigned char* uni = smem + L.uni;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int WR = p.W + p.R;
+  const int s0 = blk * p.P;                 // first step of the block within the chunk
+  if (s0 >= tlen) return;
+  const int np = min(p.P, tlen - s0);
+  const int nent = np * WR;
+
+  if (io.mode != 2) {
+    // staircase tables: row a holds columns b < min(k, n_sel / (a+1))
+    if (tid == 0) {
+      int oc = 0, of = 0, prev = -1;
+      for (int a = 0; a < p.k; ++a) {
+        const int bm = min(p.k, p.W / (a + 1));
+        for (int b = 0; b < bm; ++b) stairW[oc++] = uint32_t(a) | (uint32_t(b) << 16);
+        if (bm < p.k && !(bm == 0 && prev == 0)) frontW[of++] = uint32_t(a) | (uint32_t(bm) << 16);
+        prev = bm;
+      }
+    } else if (tid == 32) {
+      int oc = 0, of = 0, prev = -1;
+      for (int a = 0; a < p.k; ++a) {
+        const int bm = min(p.k, p.R / (a + 1));
+        for (int b = 0; b < bm; ++b) stairR[oc++] = uint32_t(a) | (uint32_t(b) << 16);
+        if (bm < p.k && !(bm == 0 && prev == 0)) frontR[of++] = uint32_t(a) | (uint32_t(bm) << 16);
+        prev = bm;
+      }
+    }
+    __syncthreads();
+    // ---- phase 1: merges, one warp per (step, side)
+    if (warp < p.merge_warps) {
+      uint64_t* h1 = reinterpret_cast<uint64_t*>(uni + L.per_warp * warp);
+      uint64_t* h2 = h1 + L.Sk;
+      uint64_t* cand = h2 + L.Sk;
+      for (int pi = warp; pi < 2 * np; pi += p.merge_warps) {
+        const int tl = pi >> 1, side = pi & 1;
+        const int tc = s0 + tl;                       // step within the chunk
+        const size_t hr = (size_t(bh) * p.Tc + tc) * 4 + side * 2;
+        const int n_sel = side ? p.R : p.W;
+        float* w_out = ent_w + tl * WR + (side ? p.W : 0);
+        uint32_t* s_out = ent_slot + tl * WR + (side ? p.W : 0);
+        merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
+                  io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
+                  side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, w_out, s_out, st,
+                  int(hr));
+        if (io.mode == 1) {
+          const size_t t = size_t(bh) * p.T + t0 + tc;
+          int32_t* oi = side ? io.out_ir : io.out_iw;
+          float* ow = side ? io.out_wr : io.out_ww;
+          for (int i = lane; i < n_sel; i += 32) {
+            oi[t * n_sel + i] = int32_t(s_out[i]);
+            ow[t * n_sel + i] = w_out[i];
+          }
+        }
+      }
+    }
+    if (io.mode == 1) return;
+  } else {
+    // ---- lists given: validate and copy
+    for (int e = tid; e < nent; e += blockDim.x) {
+      const int tl = e / WR, j = e - tl * WR;
+      const size_t t = size_t(bh) * p.T + t0 + s0 + tl;
+      int32_t s;
+      float w;
+      if (j < p.W) { s = io.in_iw[t * p.W + j]; w = io.in_ww[t * p.W + j]; }
+      else { s = io.in_ir[t * p.R + (j - p.W)]; w = io.in_wr[t * p.R + (j - p.W)]; }
+      if (s < 0 || (long long)s >= p.N) {
+        dev_flag(st, SDM_DEV_BAD_INDEX, int(t));
+        ent_slot[e] = kInvalid;
+      } else {
+        ent_slot[e] = uint32_t(s);
+      }
+      ent_w[e] = w;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 2: plan.  Hash table of the block's slots -> used once or more.
+  uint32_t* hkey = reinterpret_cast<uint32_t*>(uni);
+  unsigned char* hflag = uni + al16(size_t(L.HS) * 4);
+  uint16_t* mlist = reinterpret_cast<uint16_t*>(uni + al16(size_t(L.HS) * 4) + al16(size_t(L.HS)));
+  const uint32_t hmask = uint32_t(L.HS - 1);
+  for (int i = tid; i < L.HS; i += blockDim.x) { hkey[i] = kEmpty; hflag[i] = 0; }
+  for (int i = tid; i <= p.G; i += blockDim.x) { cnt_s[i] = 0; cnt_m[i] = 0; fill[i] = 0; }
+  if (tid == 0) misc[0] = 0;
+  __syncthreads();
+  for (int e = tid; e < nent; e += blockDim.x) {
+    const uint32_t s = ent_slot[e];
+    if (s == kInvalid) continue;
+    uint32_t h = mix32(s) & hmask;
+    for (;;) {
+      const uint32_t old = atomicCAS(&hkey[h], kEmpty, s);
+      if (old == kEmpty) break;
+      if (old == s) { hflag[h] = 1; break; }
+      h = (h + 1) & hmask;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < nent; e += blockDim.x) {
+    const uint32_t s = ent_slot[e];
+    if (s == kInvalid) continue;
+    uint32_t h = mix32(s) & hmask;
+    while (hkey[h] != s) h = (h + 1) & hmask;
+    const int part = slot_part(s, p.G);
+    if (hflag[h]) {
+      mlist[atomicAdd(&misc[0], 1)] = uint16_t(e);
+      atomicAdd(&cnt_m[part], 1);
+    } else {
+      atomicAdd(&cnt_s[part], 1);
+    }
+  }
+  __syncthreads();
+  const int n_multi = misc[0];
+  if (tid == 0) {
+    int acc = 0, macc = 0;
+    for (int g = 0; g < p.G; ++g) {
+      base[g] = acc;
+      mbase[g] = macc;
+      acc += cnt_s[g] + cnt_m[g];
+      macc += cnt_m[g];
+    }
+    base[p.G] = acc;
+  }
+  // sort the multi-use entries by (part, slot, entry) -- ascending bitonic
+  {
+    const int S = n_multi > 1 ? p2(n_multi) : 1;
+    for (int i = n_multi + tid; i < S; i += blockDim.x) mlist[i] = 0xffff;
+    __syncthreads();
+    auto mkey = [&](uint16_t e) -> uint64_t {
+      if (e == 0xffff) return ~uint64_t(0);
+      const uint32_t s = ent_slot[e];
+      return (uint64_t(slot_part(s, p.G)) << 46) | (uint64_t(s) << 14) | uint64_t(e);
+    };
+    for (int size = 2; size <= S; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < (S >> 1); i += blockDim.x) {
+          const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
+          const int hi = lo + stride;
+          const uint16_t x = mlist[lo], y = mlist[hi];
+          const uint64_t kx = mkey(x), ky = mkey(y);
+          const bool asc = (lo & size) == 0;
+          if (asc ? (kx > ky) : (kx < ky)) { mlist[lo] = y; mlist[hi] = x; }
+        }
+        __syncthreads();
+      }
+    }
+  }
+  __syncthreads();
+  int4* rec = io.rec + (size_t(bh) * p.nblk + blk) * p.E;
+  auto meta_of = [&](int e) -> int {
+    const int tl = e / WR;
+    return (tl << 1) | ((e - tl * WR) >= p.W ? 1 : 0);
+  };
+  for (int e = tid; e < nent; e += blockDim.x) {
+    const uint32_t s = ent_slot[e];
+    if (s == kInvalid) continue;
+    uint32_t h = mix32(s) & hmask;
+    while (hkey[h] != s) h = (h + 1) & hmask;
+    if (hflag[h]) continue;
+    const int part = slot_part(s, p.G);
+    const int pos = base[part] + atomicAdd(&fill[part], 1);
+    rec[pos] = make_int4(int(s), meta_of(e), __float_as_int(ent_w[e]), 1);
+  }
+  for (int i = tid; i < n_multi; i += blockDim.x) {
+    const int e = mlist[i];
+    const uint32_t s = ent_slot[e];
+    const int part = slot_part(s, p.G);
+    const int pos = base[part] + cnt_s[part] + (i - mbase[part]);
+    int len = 0;
+    if (i == 0 || ent_slot[mlist[i - 1]] != s) {
+      int j = i + 1;
+      while (j < n_multi && ent_slot[mlist[j]] == s) ++j;
+      len = j - i;
+    } else if (meta_of(mlist[i - 1]) == meta_of(e)) {
+      dev_flag(st, SDM_DEV_BAD_LIST, int(size_t(bh) * p.T + t0 + s0 + e / WR));
+    }
+    rec[pos] = make_int4(int(s), meta_of(e), __float_as_int(ent_w[e]), len);
+  }
+  int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (p.G + 1);
+  for (int g = tid; g <= p.G; g += blockDim.x) roff[g] = base[g];
+  // the recurrence accumulates o with atomics when a head has several parts
+  if (p.G > 1) {
+    float4* o4 = reinterpret_cast<float4*>(io.o + (size_t(bh) * p.T + t0 + s0) * p.dv);
+    const int n4 = np * p.dv / 4;
+    for (int i = tid; i < n4; i += blockDim.x) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+cudaError_t launch_merge_plan(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
+                              cudaStream_t s) {
+  const size_t smem = merge_smem_bytes(p, p.merge_warps);
+  cudaError_t e = cudaFuncSetAttribute(k_merge_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  const int nb = (tlen + p.P - 1) / p.P;
+  dim3 grid(nb, p.BH);
+  k_merge_plan<<<grid, kMergeThreads, smem, s>>>(p, io, t0, tlen, st);
+  return cudaGetLastError();
+}
+
+}  // namespace sdm

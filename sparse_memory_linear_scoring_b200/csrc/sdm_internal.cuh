@@ -1,0 +1,150 @@
+// sdm_internal.cuh -- shared definitions of the CUDA path (not part of the C ABI).
+//
+// The forward pass is split into three kernel families, launched per time
+// chunk on the caller's stream:
+//   1. scoring + per-half candidate lists   (score_simt.cu, score_tc.cu)
+//   2. merge of the two halves into the top-W / top-R lists, softmax weights,
+//      and the write/read plan of the recurrence           (merge_plan.cu)
+//   3. the gated delta recurrence over the slot table     (recur.cu)
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sdm.h"
+
+namespace sdm {
+
+// Fixed launch targets (depend on nothing but the problem sizes, so the
+// workspace size is a function of the dims alone).
+constexpr int kTargetCtas = 296;        // 2 x 148 SMs of a B200
+constexpr int kMaxParts = 64;           // slot parts per head in the recurrence
+constexpr int kMaxBlockEntries = 8192;  // list entries per (head, block) in a plan
+constexpr size_t kChunkBudget = size_t(1) << 30;  // workspace bytes per time chunk
+constexpr int kMergeThreads = 256;
+constexpr int kRecurThreads = 256;
+
+// Everything the kernels need to know about one call.
+struct Plan {
+  int B, H, T, dqk, dh, dv, n, k, W, R, dtype;
+  int BH;
+  long long N;
+  int tc;      // 1: tensor-core scoring, 0: SIMT scoring
+  int C;       // survivor capacity per half-row
+  int Tc;      // steps per chunk
+  int nchunks;
+  int P;       // steps per plan block
+  int nblk;    // plan blocks per chunk
+  int E;       // list entries per plan block = P * (W + R)
+  int G;       // slot parts per head
+  int ncW, nfW, ncR, nfR;  // staircase / frontier sizes of the merge
+  int merge_warps;         // warps doing merges inside a merge_plan CTA
+  size_t merge_smem, recur_smem, score_smem;
+  // workspace byte offsets
+  size_t off_status, off_cnt, off_surv, off_redo, off_rec, off_roff, total;
+};
+
+// Workspace status words.
+struct DevStatus {
+  int32_t flags;  // SDM_DEV_* bits
+  int32_t info;   // first offending index, -1 if none
+  int32_t redo;   // number of half-rows queued for the exact SIMT path
+  int32_t pad[13];
+};
+
+int make_plan(const sdm_dims* d, Plan* p);  // SDM_OK or an error code
+
+// ---- device helpers ---------------------------------------------------------
+__device__ __forceinline__ uint32_t f2ord(float v) {
+  if (v == 0.0f) v = 0.0f;  // -0 and +0 compare equal: give them one key
+  uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float ord2f(uint32_t o) {
+  uint32_t b = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
+  return __uint_as_float(b);
+}
+// Larger key = larger value, then smaller index.
+__device__ __forceinline__ uint64_t make_key(float v, uint32_t idx) {
+  return (uint64_t(f2ord(v)) << 32) | uint64_t(~idx);
+}
+__device__ __forceinline__ float key_val(uint64_t key) { return ord2f(uint32_t(key >> 32)); }
+__device__ __forceinline__ uint32_t key_idx(uint64_t key) { return ~uint32_t(key); }
+
+__device__ __forceinline__ uint32_t mix32(uint32_t x) {
+  x ^= x >> 16; x *= 0x85ebca6bu;
+  x ^= x >> 13; x *= 0xc2b2ae35u;
+  x ^= x >> 16;
+  return x;
+}
+// Which part (recurrence CTA) of a head owns a slot.
+__device__ __forceinline__ int slot_part(uint32_t slot, int G) {
+  return int(mix32(slot ^ 0x9e3779b9u) % uint32_t(G));
+}
+
+__device__ __forceinline__ void dev_flag(DevStatus* st, int bits, int info) {
+  atomicOr(&st->flags, bits);
+  atomicCAS(&st->info, -1, info);
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+// Descending bitonic sort of S (power of two) 64-bit keys in shared memory by
+// one warp.
+__device__ __forceinline__ void warp_sort_desc(uint64_t* a, int S) {
+  const int lane = threadIdx.x & 31;
+  for (int size = 2; size <= S; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = lane; i < (S >> 1); i += 32) {
+        const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
+        const int hi = lo + stride;
+        const uint64_t x = a[lo], y = a[hi];
+        const bool desc = (lo & size) == 0;
+        if (desc ? (x < y) : (x > y)) { a[lo] = y; a[hi] = x; }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+inline int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// ---- launchers (one per kernel family) --------------------------------------
+cudaError_t launch_init(const Plan& p, DevStatus* st, cudaStream_t s);
+cudaError_t launch_score_simt(const Plan& p, const void* q, const void* k, const void* C1,
+                              const void* C2, int t0, int tlen, const int* rows,
+                              const DevStatus* st_rows, int* surv_cnt, uint2* surv,
+                              DevStatus* st, cudaStream_t s);
+cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const void* C1,
+                            const void* C2, int t0, int tlen, int* surv_cnt, uint2* surv,
+                            int* redo_rows, DevStatus* st, cudaStream_t s);
+bool score_tc_supported(const sdm_dims* d);
+
+struct MergeIO {
+  // mode 0: survivors -> plan;  1: survivors -> lists;  2: lists -> plan
+  int mode;
+  const int* surv_cnt;
+  const uint2* surv;
+  const int32_t* in_iw; const float* in_ww; const int32_t* in_ir; const float* in_wr;
+  int32_t* out_iw; float* out_ww; int32_t* out_ir; float* out_wr;
+  int4* rec;
+  int* roff;
+  float* o;
+};
+cudaError_t launch_merge_plan(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
+                              cudaStream_t s);
+
+cudaError_t launch_recur(const Plan& p, const void* v, const float* alpha, const float* beta,
+                         float* M, float* o, const int4* rec, const int* roff, int t0, int tlen,
+                         DevStatus* st, cudaStream_t s);
+
+}  // namespace sdm

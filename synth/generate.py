@@ -6,7 +6,7 @@ on a CUDA device, without generating the rest.  The generator is written with
 torch int64 tensor arithmetic (two's-complement wrap-around gives the same bits
 as uint64 arithmetic), so one definition serves both devices.
 
-Recipe (readings of the workload descriptions, "Input recipe"):
+Recipe (readings of the workload descriptions where they are silent):
   * splitmix64: state_i = key + (i+1)*0x9E3779B97F4A7C15, output = mix(state_i)
     with the published splitmix64 finaliser (Steele, Lea, Flood 2014).
   * U(0,1): ((z >> 11) + 0.5) / 2^53, never 0 or 1.
@@ -192,11 +192,13 @@ def gen_head_inputs(cfg: SDMConfig, b: int, h: int, seed: int = 0,
 
 
 def gen_inputs(cfg: SDMConfig, seed: int = 0, device: str = 'cpu',
-               t_end: Optional[int] = None, with_m0: bool = True) -> Dict[str, torch.Tensor]:
+               t_end: Optional[int] = None, with_m0: bool = True,
+               b0: int = 0) -> Dict[str, torch.Tensor]:
     """All inputs, full layout: q,k [B,H,T,d_qk], v [B,H,T,d_v], alpha,beta [B,H,T],
-    C1,C2 [H,n,d_h], M0 [B,H,N,d_v] (float32 values)."""
-    return _gen(cfg, list(range(cfg.B)), list(range(cfg.H)), seed, device, t_end, with_m0,
-                squeeze=False)
+    C1,C2 [H,n,d_h], M0 [B,H,N,d_v] (float32 values).  b0 offsets the batch
+    index (a shard [b0, b0+B) of a larger batch)."""
+    return _gen(cfg, list(range(b0, b0 + cfg.B)), list(range(cfg.H)), seed, device, t_end,
+                with_m0, squeeze=False)
 
 
 def _gen(cfg, bs, hs, seed, device, t_end, with_m0, squeeze):

@@ -1,0 +1,161 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+seeded synthetic workloads, element by element.
+
+Bars: selected slot sets equal except at oracle-flagged near-ties (< 0.1% of
+selections); o and M within 1e-4 relative (max abs error over max abs value,
+per head); heads with a flagged selection difference are also compared after
+feeding the oracle's lists to the recurrence kernel (sdm_recur), so a
+legitimate tie flip is not scored as numeric error."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_memory_linear_scoring_b200 as sdm
+from gpu_util import (READ_BITS, REL_TOL, WRITE_BITS, compare_lists, gpu_forward, gpu_select,
+                      head_rel_err, np_inputs, oracle_full, to_device)
+from synth import config, gen_inputs
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _status_clean():
+    st, info = sdm.device_status()
+    assert st == 0, "device status %d (info %d)" % (st, info)
+
+
+def _check_forward(cfg, inp, ref, d=None):
+    d = d if d is not None else to_device(inp, cfg)
+    o, M = gpu_forward(d, cfg)
+    iw, ww, ir, wr = gpu_select(d, cfg)
+    torch.cuda.synchronize()
+    _status_clean()
+    _, same_w = compare_lists(iw.cpu().numpy(), ww.cpu().numpy(), ref["idx_w"], ref["w_w"],
+                              ref["flags"], WRITE_BITS, "write lists")
+    _, same_r = compare_lists(ir.cpu().numpy(), wr.cpu().numpy(), ref["idx_r"], ref["w_r"],
+                              ref["flags"], READ_BITS, "read lists")
+    clean = same_w.all(axis=-1) & same_r.all(axis=-1)          # [B,H]
+    eo = head_rel_err(o.cpu().numpy(), ref["o"])
+    eM = head_rel_err(M.cpu().numpy(), ref["M"])
+    assert (eo[clean] <= REL_TOL).all(), eo
+    assert (eM[clean] <= REL_TOL).all(), eM
+    # the recurrence alone, fed the oracle's lists
+    M2 = d["M"].clone()
+    o2 = sdm.recur(d["v"], d["alpha"], d["beta"],
+                   torch.from_numpy(ref["idx_w"].astype(np.int32)).cuda(),
+                   torch.from_numpy(ref["w_w"].astype(np.float32)).cuda(),
+                   torch.from_numpy(ref["idx_r"].astype(np.int32)).cuda(),
+                   torch.from_numpy(ref["w_r"].astype(np.float32)).cuda(), M2,
+                   d_qk=cfg.d_qk, n_sub=cfg.n_sub, topk=cfg.k)
+    torch.cuda.synchronize()
+    _status_clean()
+    assert (head_rel_err(o2.cpu().numpy(), ref["o"]) <= REL_TOL).all()
+    assert (head_rel_err(M2.cpu().numpy(), ref["M"]) <= REL_TOL).all()
+    return o, M
+
+
+def test_golden_hand_example():
+    with open(os.path.join(GOLDEN, "hand_two_steps.json")) as f:
+        g = json.load(f)
+    dm = g["dims"]
+    dev = "cuda"
+    f32 = dict(dtype=torch.float32, device=dev)
+    # d_v = 2 is below the kernels' 4-float row granule: pad rows with zeros
+    pad = lambda a: torch.nn.functional.pad(torch.tensor(a, **f32), (0, 2))
+    q = torch.tensor(g["q"], **f32)[None, None].contiguous()
+    k = torch.tensor(g["k"], **f32)[None, None].contiguous()
+    v = pad(g["v"])[None, None].contiguous()
+    al = torch.tensor(g["alpha"], **f32)[None, None].contiguous()
+    be = torch.tensor(g["beta"], **f32)[None, None].contiguous()
+    C1 = torch.tensor(g["C1"], **f32)[None].contiguous()
+    C2 = torch.tensor(g["C2"], **f32)[None].contiguous()
+    M = pad(g["M0"])[None, None].contiguous()
+    o = sdm.forward(q, k, v, al, be, C1, C2, M, topk=dm["k"], W=dm["W"], R=dm["R"])
+    iw, ww, ir, wr = sdm.select(q, k, C1, C2, topk=dm["k"], W=dm["W"], R=dm["R"])
+    torch.cuda.synchronize()
+    _status_clean()
+    e = g["expect"]
+    assert iw[0, 0].cpu().tolist() == e["idx_w"]
+    assert ir[0, 0].cpu().tolist() == e["idx_r"]
+    np.testing.assert_allclose(ww[0, 0].cpu().numpy(), np.array(e["w_w"]), rtol=1e-6)
+    np.testing.assert_allclose(o[0, 0, :, :2].cpu().numpy(), np.array(e["o"]), rtol=1e-6)
+    np.testing.assert_allclose(M[0, 0, :, :2].cpu().numpy(), np.array(e["M"]), rtol=1e-6)
+    assert (o[0, 0, :, 2:] == 0).all() and (M[0, 0, :, 2:] == 0).all()
+
+
+@pytest.mark.parametrize("ci", [0, 1, 2])
+def test_forward_parity_full(ci):
+    cfg = config(ci)
+    inp = gen_inputs(cfg)
+    ref = oracle_full(inp, cfg, lists=True)
+    o, M = _check_forward(cfg, inp, ref)
+    # the unselected rows are bit-identical to M_0
+    written = np.zeros((cfg.B, cfg.H, cfg.N), dtype=bool)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            written[b, h, np.unique(ref["idx_w"][b, h])] = True
+    M0 = inp["M0"].numpy()
+    Mg = M.cpu().numpy()
+    assert np.array_equal(Mg[~written], M0[~written])
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=1), dict(T=2), dict(T=97), dict(T=1000), dict(W=1, R=1), dict(k=2, W=4, R=3),
+    dict(W=64, R=1), dict(n_sub=8, k=8, W=64, R=64, T=64),
+])
+def test_forward_parity_shapes(shape):
+    """Ragged blocks, single steps, W = k^2 (every candidate), W = R = 1."""
+    base = config(1).with_(B=1, H=2, T=300, n_sub=64, k=16, W=32, R=32, m0_sd=0.5)
+    cfg = base.with_(**shape)
+    inp = gen_inputs(cfg)
+    ref = oracle_full(inp, cfg, lists=True)
+    _check_forward(cfg, inp, ref)
+
+
+def test_fp32_wide_rows():
+    cfg = config(0).with_(B=2, H=3, T=200, d_v=128, d_qk=24, n_sub=16, k=6, W=20, R=12,
+                          m0_sd=1.0)
+    inp = gen_inputs(cfg)
+    ref = oracle_full(inp, cfg, lists=True)
+    _check_forward(cfg, inp, ref)
+
+
+def test_empty_sequence():
+    cfg = config(0).with_(T=0)
+    inp = gen_inputs(cfg)
+    d = to_device(inp, cfg)
+    M = d["M"].clone()
+    o = sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], M,
+                    topk=cfg.k, W=cfg.W, R=cfg.R)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and torch.equal(M, d["M"])
+
+
+def test_recur_flags_bad_lists():
+    """sdm_recur records out-of-range and repeated slots in the device status."""
+    cfg = config(0).with_(T=8)
+    inp = gen_inputs(cfg)
+    d = to_device(inp, cfg)
+    ref = oracle_full(inp, cfg, lists=True)
+    iw = torch.from_numpy(ref["idx_w"].astype(np.int32)).cuda()
+    ww = torch.from_numpy(ref["w_w"].astype(np.float32)).cuda()
+    ir = torch.from_numpy(ref["idx_r"].astype(np.int32)).cuda()
+    wr = torch.from_numpy(ref["w_r"].astype(np.float32)).cuda()
+    bad = iw.clone()
+    bad[0, 0, 3, 1] = cfg.N + 5
+    M = d["M"].clone()
+    sdm.recur(d["v"], d["alpha"], d["beta"], bad, ww, ir, wr, M, d_qk=cfg.d_qk, n_sub=cfg.n_sub,
+              topk=cfg.k)
+    st, info = sdm.device_status()
+    assert st & 1 and info == 3
+    rep = iw.clone()
+    rep[0, 0, 5, 2] = rep[0, 0, 5, 1]
+    sdm.recur(d["v"], d["alpha"], d["beta"], rep, ww, ir, wr, d["M"].clone(), d_qk=cfg.d_qk,
+              n_sub=cfg.n_sub, topk=cfg.k)
+    st, info = sdm.device_status()
+    assert st & 8 and info == 5
