@@ -173,6 +173,9 @@ def run_sdm(args, cfg, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     nph = 4 * plan["chunks"]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(nph)]
+    for e in ev:          # torch creates the CUDA event on its first record
+        e.record()
+    torch.cuda.synchronize(dev)
 
     def step(events=None):
         sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], M,

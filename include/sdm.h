@@ -29,7 +29,8 @@
  *      o      [B][H][T][d_v]    float32
  *      idx_w / w_w [B][H][T][W] int32 / float32 (idx_r / w_r likewise with R)
  *  - Every device pointer must be 16-byte aligned; outputs must not alias
- *    inputs or each other.
+ *    inputs or each other.  With T == 0 nothing is enqueued and no pointer is
+ *    read (empty tensors may pass NULL).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work
  *    is enqueued on it and the call returns without waiting; results are
  *    valid after the stream is synchronised.

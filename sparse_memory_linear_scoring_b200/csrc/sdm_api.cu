@@ -200,6 +200,7 @@ static int forward_impl(const void* q, const void* k, const void* v, const float
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
+  if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
   rc = check_ptrs({q, k, v, alpha, beta, C1, C2, M_inout, o_out, workspace});
   if (rc != SDM_OK) return rc == SDM_ERR_NULL && !workspace ? SDM_ERR_WORKSPACE : rc;
   if (ws_bytes < p.total) return SDM_ERR_WORKSPACE;
@@ -267,6 +268,7 @@ extern "C" int sdm_select(const void* q, const void* k, const void* C1, const vo
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
+  if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
   rc = check_ptrs({q, k, C1, C2, idx_w, w_w, idx_r, w_r, workspace});
   if (rc != SDM_OK) return rc == SDM_ERR_NULL && !workspace ? SDM_ERR_WORKSPACE : rc;
   if (ws_bytes < p.total) return SDM_ERR_WORKSPACE;
@@ -295,6 +297,7 @@ extern "C" int sdm_recur(const void* v, const float* alpha, const float* beta,
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
+  if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
   rc = check_ptrs({v, alpha, beta, idx_w, w_w, idx_r, w_r, M_inout, o_out, workspace});
   if (rc != SDM_OK) return rc == SDM_ERR_NULL && !workspace ? SDM_ERR_WORKSPACE : rc;
   if (ws_bytes < p.total) return SDM_ERR_WORKSPACE;
