@@ -81,7 +81,8 @@ enum {
   SDM_ERR_WORKSPACE = 4,   /* workspace missing or smaller than sdm_workspace_bytes */
   SDM_ERR_UNSUPPORTED = 5, /* valid sizes this build has no kernel for */
   SDM_ERR_CUDA = 6,        /* a CUDA call failed while enqueueing */
-  SDM_ERR_DEVICE = 7       /* a kernel's own check fired (see sdm_get_device_status) */
+  SDM_ERR_DEVICE = 7,      /* a kernel's own check fired (see sdm_get_device_status) */
+  SDM_ERR_SCRATCH_LIMIT = 8 /* sdm_forward_noalloc: problem needs more than its 64 MiB scratch */
 };
 
 /* Device status bits recorded by the kernels (sdm_get_device_status). */
@@ -149,6 +150,31 @@ SDM_API int sdm_forward_timed(const void* q, const void* k, const void* v, const
                               const float* beta, const void* C1, const void* C2, float* M_inout,
                               float* o_out, const sdm_dims* dims, void* workspace,
                               size_t ws_bytes, void* stream, void* const* events, int n_events);
+
+/*
+ * sdm_forward without a workspace argument, for callers that cannot allocate
+ * device memory: a plugin whose host framework owns the whole device-memory
+ * budget and forbids allocations on the execution path, or a latency-critical
+ * loop that cannot pay for the device synchronisation cudaMalloc / cudaFree
+ * imply.  The pages have no counterpart; this is an interface convenience.
+ *
+ * Its scratch is one file-scope device array of 64 MiB that every GPU loading
+ * this library holds until the process exits.  Problems whose
+ * sdm_workspace_bytes(dims) exceeds 64 MiB are rejected with
+ * SDM_ERR_SCRATCH_LIMIT before anything is enqueued.  Runs on the current
+ * device; `stream` must belong to it.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Every call shares the one
+ * array and it keeps the last call's contents (nothing in it needs to start
+ * at zero), so calls that overlap on the GPU race: serialise them (one stream,
+ * or events).  The kernels' status word is not readable through this entry
+ * point.  Allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * call).  Results and other return codes as sdm_forward.
+ */
+SDM_API int sdm_forward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
+                                const float* beta, const void* C1, const void* C2,
+                                float* M_inout, float* o_out, const sdm_dims* dims,
+                                void* stream);
 
 /*
  * How the library will run `dims` (host only, no GPU work).  Writes up to n

@@ -346,6 +346,7 @@ extern "C" const char* sdm_status_string(int status) {
     case SDM_ERR_UNSUPPORTED: return "valid sizes without a kernel in this build";
     case SDM_ERR_CUDA: return "a CUDA call failed while enqueueing";
     case SDM_ERR_DEVICE: return "a kernel's own check fired";
+    case SDM_ERR_SCRATCH_LIMIT: return "problem needs more than the 64 MiB static scratch";
     default: return "unknown status";
   }
 }
