@@ -39,6 +39,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sdm", "reference"], default="sdm")
     ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--T", type=int, default=0,
+                    help="override the number of steps (small profiling captures only)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -365,6 +367,8 @@ def main():
     args = parse()
     from synth import config
     cfg = config(args.config)
+    if args.T > 0:
+        cfg = cfg.with_(T=args.T)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -7,9 +7,9 @@
 // ordered by (float32 sum descending, slot ascending).  Item 3 weights: w =
 // softmax over the W selected write scores, u = softmax over the R read scores.
 //
-// Merge (one warp per (step, side)): sort each half's survivors, evaluate the
+// Merge (one warp per (step, side)): the half lists arrive sorted; evaluate the
 // "staircase" candidates (a, b) with (a+1)(b+1) <= n_sel (a, b = ranks in the
-// two halves), sort them, and take the first n_sel.  This is exact when every
+// two halves) and select the n_sel best by quickselect.  This is exact when every
 // candidate outside the staircase scores strictly below the n_sel-th: the
 // largest outside score is attained on the staircase's frontier (row a, column
 // bmax(a)), since sums fall along each row; if the frontier check fails, an
@@ -32,7 +32,7 @@ constexpr uint32_t kInvalid = 0xffffffffu;
 
 struct MergeLayout {
   size_t ent_slot, ent_w, stair, misc, uni, total;
-  int Sk, Sc, HS, warps;
+  int Sk, Sc, Ss, HS, warps;
   size_t per_warp, phase2;
 };
 
@@ -46,7 +46,8 @@ __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15)
 
 __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   MergeLayout L;
-  L.Sk = p2(p.C);
+  L.Sk = p2(p.k);
+  L.Ss = p2(p.W > p.R ? p.W : p.R);
   L.Sc = p2(p.ncW > p.ncR ? p.ncW : p.ncR);
   L.HS = p2(2 * p.E);
   L.warps = warps;
@@ -56,7 +57,7 @@ __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR) * 4);
   L.misc = o; o = al16(o + size_t(5 * (kMaxParts + 1) + 8) * 4);
   L.uni = o;
-  L.per_warp = size_t(2 * L.Sk + L.Sc) * 8;
+  L.per_warp = size_t(2 * L.Sk + L.Sc + L.Ss + 32) * 8;
   L.phase2 = al16(size_t(L.HS) * 4) + al16(size_t(L.HS)) + al16(size_t(p2(p.E)) * 2);
   const size_t ph1 = L.per_warp * warps;
   o += (ph1 > L.phase2 ? ph1 : L.phase2);
@@ -111,66 +112,169 @@ __device__ void merge_full(const uint64_t* h1, const uint64_t* h2, int k, int n,
   warp_sort_desc(cand, S);
 }
 
-// Sorted top-k of one half's survivors into h[0..k); returns false when the
-// survivor count is out of range.
-__device__ bool half_topk(const uint2* sv, int cnt, int k, int C, uint64_t* h) {
-  const int lane = threadIdx.x & 31;
-  if (cnt < k || cnt > C) return false;
-  const int S = p2(cnt);
-  for (int i = lane; i < S; i += 32)
-    h[i] = (i < cnt) ? make_key(__uint_as_float(sv[i].x), sv[i].y) : uint64_t(0);
-  __syncwarp();
-  warp_sort_desc(h, S);
-  return true;
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
+// Descending bitonic sort of one 64-bit key per lane across the warp.
+__device__ __forceinline__ uint64_t warp_sort32_desc(uint64_t x) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t y = __shfl_xor_sync(0xffffffffu, x, stride);
+      const bool desc = (lane & size) == 0 || size == 32;
+      const bool lower = (lane & stride) == 0;
+      x = (lower == desc) ? (x > y ? x : y) : (x < y ? x : y);
+    }
+  }
+  return x;
+}
+
+// The r-th largest (1-based) of the nc distinct, nonzero keys in cand[]:
+// quickselect with pseudo-random pivots over the shrinking interval (L, U],
+// finished by a 32-key sort.  tmp holds 32 keys.
+__device__ uint64_t warp_select(const uint64_t* cand, int nc, int r, uint64_t* tmp) {
+  const int lane = threadIdx.x & 31;
+  uint64_t L = 0, U = ~uint64_t(0);
+  int above = 0;  // keys > U
+  uint32_t seed = 0x9e3779b9u;
+  for (int iter = 0; iter < 4096; ++iter) {
+    int act = 0;
+    for (int i = lane; i < nc; i += 32) {
+      const uint64_t x = cand[i];
+      act += (x > L) & (x <= U);
+    }
+    int incl = act;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+    if (tot <= 32) {
+      int base = 0;
+      for (int i0 = 0; i0 < nc; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t x = i < nc ? cand[i] : 0;
+        const bool a = (i < nc) && (x > L) && (x <= U);
+        const unsigned m = __ballot_sync(0xffffffffu, a);
+        if (a) tmp[base + __popc(m & lanemask_lt())] = x;
+        base += __popc(m);
+      }
+      __syncwarp();
+      uint64_t mine = lane < tot ? tmp[lane] : 0;
+      __syncwarp();
+      mine = warp_sort32_desc(mine);
+      return __shfl_sync(0xffffffffu, mine, r - above - 1);
+    }
+    seed = seed * 1664525u + 1013904223u;
+    const int j = int((uint64_t(seed >> 8) * uint64_t(tot)) >> 24);  // [0, tot)
+    const int owner = __ffs(__ballot_sync(0xffffffffu, incl > j)) - 1;
+    uint64_t piv = 0;
+    if (lane == owner) {
+      int want = j - (incl - act);
+      for (int i = lane; i < nc; i += 32) {
+        const uint64_t x = cand[i];
+        if ((x > L) && (x <= U)) {
+          if (want == 0) { piv = x; break; }
+          --want;
+        }
+      }
+    }
+    piv = __shfl_sync(0xffffffffu, piv, owner);
+    int ge = 0;
+    for (int i = lane; i < nc; i += 32) {
+      const uint64_t x = cand[i];
+      ge += (x >= piv) & (x <= U);
+    }
+    ge = __reduce_add_sync(0xffffffffu, ge);
+    const int G = above + ge;
+    if (G == r) return piv;
+    if (G > r) {
+      L = piv;
+    } else {
+      U = piv - 1;
+      above = G;
+    }
+  }
+  return 0;  // not reached: every iteration removes the pivot from (L, U]
+}
+
+// Merge of one (step, side): sorted half lists (first k entries of each
+// survivor list) -> the n_sel selected slots and their softmax weights.
+// Selection order is unspecified unless `sorted` is set (then rank order).
 __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
                           int n_sel, const uint32_t* stair, int nc, const uint32_t* front, int nf,
-                          uint64_t* h1, uint64_t* h2, uint64_t* cand, float* w_out,
-                          uint32_t* slot_out, DevStatus* st, int info) {
+                          uint64_t* h1, uint64_t* h2, uint64_t* cand, uint64_t* sel,
+                          uint64_t* tmp, bool sorted, float* w_out, uint32_t* slot_out,
+                          DevStatus* st, int info) {
   const int lane = threadIdx.x & 31;
-  const bool ok1 = half_topk(sv1, c1, p.k, p.C, h1);
-  const bool ok2 = half_topk(sv2, c2, p.k, p.C, h2);
-  if (!ok1 || !ok2) {
+  if (c1 < p.k || c1 > p.C || c2 < p.k || c2 > p.C) {
     if (lane == 0) dev_flag(st, SDM_DEV_CAPACITY, info);
     for (int i = lane; i < n_sel; i += 32) { w_out[i] = 0.f; slot_out[i] = kInvalid; }
     __syncwarp();
     return;
   }
-  const uint32_t n = uint32_t(p.n);
-  const int Sc = p2(nc);
-  for (int i = lane; i < Sc; i += 32) {
-    uint64_t key = 0;
-    if (i < nc) {
-      const uint32_t ab = stair[i];
-      const int a = ab & 0xffff, b = ab >> 16;
-      const float v = key_val(h1[a]) + key_val(h2[b]);
-      key = make_key(v, key_idx(h1[a]) * n + key_idx(h2[b]));
-    }
-    cand[i] = key;
+  for (int i = lane; i < p.k; i += 32) {
+    const uint2 a = sv1[i], b = sv2[i];
+    h1[i] = make_key(__uint_as_float(a.x), a.y);
+    h2[i] = make_key(__uint_as_float(b.x), b.y);
   }
   __syncwarp();
-  warp_sort_desc(cand, Sc);
-  // frontier check: every candidate outside the staircase must score strictly
-  // below the n_sel-th staircase candidate
-  const uint32_t tau = uint32_t(cand[n_sel - 1] >> 32);
+  const uint32_t n = uint32_t(p.n);
+  for (int i = lane; i < nc; i += 32) {
+    const uint32_t ab = stair[i];
+    const int a = ab & 0xffff, b = ab >> 16;
+    const float v = key_val(h1[a]) + key_val(h2[b]);
+    cand[i] = make_key(v, key_idx(h1[a]) * n + key_idx(h2[b]));
+  }
+  __syncwarp();
+  const uint64_t kth = warp_select(cand, nc, n_sel, tmp);
+  // every candidate outside the staircase must score strictly below the kth
+  const uint32_t tau = uint32_t(kth >> 32);
   bool bad = false;
   for (int i = lane; i < nf; i += 32) {
     const uint32_t ab = front[i];
     const int a = ab & 0xffff, b = ab >> 16;
     bad |= f2ord(key_val(h1[a]) + key_val(h2[b])) >= tau;
   }
-  if (__any_sync(0xffffffffu, bad)) merge_full(h1, h2, p.k, p.n, n_sel, cand);
-  // softmax over the selected float32 scores
-  const float m = key_val(cand[0]);
+  bool is_sorted = false;
+  if (__any_sync(0xffffffffu, bad)) {
+    merge_full(h1, h2, p.k, p.n, n_sel, cand);
+    for (int i = lane; i < n_sel; i += 32) sel[i] = cand[i];
+    is_sorted = true;
+  } else {
+    int base = 0;
+    for (int i0 = 0; i0 < nc; i0 += 32) {
+      const int i = i0 + lane;
+      const uint64_t x = i < nc ? cand[i] : 0;
+      const bool take = (i < nc) && x >= kth;
+      const unsigned m = __ballot_sync(0xffffffffu, take);
+      if (take) sel[base + __popc(m & lanemask_lt())] = x;
+      base += __popc(m);
+    }
+  }
+  __syncwarp();
+  if (sorted && !is_sorted) {
+    const int S = p2(n_sel);
+    for (int i = n_sel + lane; i < S; i += 32) sel[i] = 0;
+    __syncwarp();
+    warp_sort_desc(sel, S);
+  }
+  // softmax over the selected float32 scores; the best candidate is (0, 0)
+  const float m = key_val(h1[0]) + key_val(h2[0]);
   float zs = 0.f;
-  for (int i = lane; i < n_sel; i += 32) zs += expf(key_val(cand[i]) - m);
+  for (int i = lane; i < n_sel; i += 32) zs += expf(key_val(sel[i]) - m);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
   const float inv = 1.f / zs;
   for (int i = lane; i < n_sel; i += 32) {
-    w_out[i] = expf(key_val(cand[i]) - m) * inv;
-    slot_out[i] = key_idx(cand[i]);
+    w_out[i] = expf(key_val(sel[i]) - m) * inv;
+    slot_out[i] = key_idx(sel[i]);
   }
   __syncwarp();
 }
@@ -227,6 +331,8 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
       uint64_t* h1 = reinterpret_cast<uint64_t*>(uni + L.per_warp * warp);
       uint64_t* h2 = h1 + L.Sk;
       uint64_t* cand = h2 + L.Sk;
+      uint64_t* sel = cand + L.Sc;
+      uint64_t* tmp = sel + L.Ss;
       for (int pi = warp; pi < 2 * np; pi += p.merge_warps) {
         const int tl = pi >> 1, side = pi & 1;
         const int tc = s0 + tl;                       // step within the chunk
@@ -236,8 +342,8 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
         uint32_t* s_out = ent_slot + tl * WR + (side ? p.W : 0);
         merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
                   io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
-                  side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, w_out, s_out, st,
-                  int(hr));
+                  side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, sel, tmp,
+                  io.mode == 1, w_out, s_out, st, int(hr));
         if (io.mode == 1) {
           const size_t t = size_t(bh) * p.T + t0 + tc;
           int32_t* oi = side ? io.out_ir : io.out_iw;

@@ -1,17 +1,510 @@
-// score_tc.cu -- tensor-core (tcgen05) sub-key scoring; filled in below.
+// score_tc.cu -- sub-key scoring on the 5th-generation tensor cores (tcgen05)
+// with a per-row threshold filter and an exact sorted top-k per half-row.
+//
+// SDM summaries (gist.science 2607.07386), "Mecanismo Central" item 2: each
+// half of k'_t / q'_t is scored against its sub-key codebook (a dense
+// contraction: tokens x d_h times d_h x n_sub) and keeps its top-k.
+//
+// One CTA = 128 tokens of one (b,h) head, one side (k' or q') and one half:
+//   warp 0      TMA producer: the 128 x d_h token tile once, then the codebook
+//               in 256-row tiles through a 2-stage shared-memory ring (128-byte
+//               swizzle, bf16, K-major);
+//   warp 1      allocates 512 TMEM columns; one lane issues
+//               tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32, M=128, N=256,
+//               K=16 steps) into two 256-column TMEM buffers;
+//   warps 2..5  epilogue, one thread per token row (TMEM lane): tcgen05.ld the
+//               row's scores, keep those above a threshold tau taken from the
+//               row's own score mean and deviation (first 512 columns), then
+//               select the exact top-k of the kept scores and write them sorted
+//               by (score desc, row asc).
+// A row whose kept count falls outside [k, capacity] (or whose scores do not
+// spread) is queued for the exact CUDA-core path instead, so the result is
+// exact for any input.  Every mbarrier wait is bounded: on a timeout the CTA
+// records SDM_DEV_TIMEOUT, stops issuing work, drains what it issued (bounded)
+// and frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <mutex>
+
 #include "sdm_internal.cuh"
 
 namespace sdm {
+namespace {
 
-bool score_tc_supported(const sdm_dims* d) { (void)d; return false; }
-int score_tc_capacity(const sdm_dims* d) { return d->k; }
-size_t score_tc_smem(const Plan& p) { (void)p; return 0; }
+constexpr int kTileM = 128;
+constexpr int kTileN = 256;
+constexpr int kKAtom = 64;           // bf16 elements per 128-byte swizzle row
+constexpr int kThreads = 192;
+constexpr int kBuckets = 64;         // final-selection buckets per row
+constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+constexpr uint32_t kATileBytes = kTileM * 128;   // one 64-column chunk of the token tile
+constexpr uint32_t kBTileBytes = kTileN * 128;   // one 64-column chunk of a codebook tile
+
+struct TcArgs {
+  Plan p;
+  int t0, tlen;
+  float z;          // threshold in deviations above the row mean (-inf: keep all)
+  uint2* surv;
+  int* cnt;
+  int* redo;
+  DevStatus* st;
+};
+
+struct TcLayout {
+  uint32_t a, b, vals, idx, hist, bars, total;
+  int nkc;
+};
+
+__host__ __device__ inline TcLayout tc_layout(const Plan& p) {
+  TcLayout L;
+  L.nkc = p.dh / kKAtom;
+  uint32_t o = 0;
+  L.a = o; o += L.nkc * kATileBytes;
+  L.b = o; o += 2 * L.nkc * kBTileBytes;
+  L.vals = o; o += uint32_t(p.C) * kTileM * 4;
+  L.idx = o; o += uint32_t(p.C) * kTileM * 2;
+  o = (o + 15) & ~15u;
+  L.hist = o; o += kBuckets * kTileM * 2;
+  o = (o + 15) & ~15u;
+  L.bars = o; o += 16 * 8;
+  L.total = o + 1024;  // slack for 1024-byte alignment of the dynamic base
+  return L;
+}
+
+// ---- PTX wrappers -------------------------------------------------------------
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false when it timed out or another role already gave up.
+__device__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (!mbar_test(b, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+// K-major, 128-byte swizzle shared-memory matrix descriptor (8-row groups
+// 1024 bytes apart).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t(1) << 16;          // leading byte offset (unused for swizzled K-major)
+  d |= uint64_t(1024 >> 4) << 32;  // stride byte offset
+  d |= uint64_t(1) << 46;          // descriptor version (sm_100)
+  d |= uint64_t(2) << 61;          // 128-byte swizzle
+  return d;
+}
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          su32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// (score desc, row asc) order on the output pairs
+__device__ __forceinline__ bool before(uint2 a, uint2 b) {
+  const float va = __uint_as_float(a.x), vb = __uint_as_float(b.x);
+  return va > vb || (va == vb && a.y < b.y);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+           const __grid_constant__ CUtensorMap mc1, const __grid_constant__ CUtensorMap mc2,
+           TcArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Plan& p = a.p;
+  const TcLayout L = tc_layout(p);
+  unsigned char* sA = smem + L.a;
+  unsigned char* sB = smem + L.b;
+  float* vals = reinterpret_cast<float*>(smem + L.vals);
+  uint16_t* idxs = reinterpret_cast<uint16_t*>(smem + L.idx);
+  uint16_t* hist = reinterpret_cast<uint16_t*>(smem + L.hist);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* full = bars;       // [2] TMA -> MMA
+  uint64_t* empty = bars + 2;  // [2] MMA -> TMA
+  uint64_t* a_full = bars + 4;
+  uint64_t* tfull = bars + 5;  // [2] MMA -> epilogue
+  uint64_t* tempty = bars + 7; // [2] epilogue -> MMA
+  uint64_t* drain = bars + 9;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, bh = blockIdx.y, side = blockIdx.z >> 1, half = blockIdx.z & 1;
+  const int h = bh % p.H;
+  const int ntiles = p.n / kTileN;
+  const int nk = p.dh / 16;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4 * 32);
+    }
+    mbar_init(a_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     su32(const_cast<uint32_t*>(tmem_slot)))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      const CUtensorMap* mx = side ? &mq : &mk;
+      const CUtensorMap* mc = half ? &mc2 : &mc1;
+      tma_prefetch(mx);
+      tma_prefetch(mc);
+      const int row0 = bh * p.T + a.t0 + tile * kTileM;
+      mbar_expect_tx(a_full, L.nkc * kATileBytes);
+      for (int kc = 0; kc < L.nkc; ++kc)
+        tma_load_2d(mx, a_full, sA + kc * kATileBytes, half * p.dh + kc * kKAtom, row0);
+      int issued = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+        mbar_expect_tx(&full[s], L.nkc * kBTileBytes);
+        for (int kc = 0; kc < L.nkc; ++kc)
+          tma_load_2d(mc, &full[s], sB + (s * L.nkc + kc) * kBTileBytes, kc * kKAtom,
+                      h * p.n + j * kTileN);
+        ++issued;
+      }
+      // on abort: let the copies already issued land before the CTA leaves
+      if (*abort_flag) {
+        volatile int never = 0;
+        mbar_wait(a_full, 0, &never);
+        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+          mbar_wait(&full[j & 1], (j >> 1) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kTileM, kTileN);
+      int issued = 0;
+      if (mbar_wait(a_full, 0, abort_flag)) {
+        for (int j = 0; j < ntiles; ++j) {
+          const int s = j & 1;
+          if (!mbar_wait(&full[s], (j >> 1) & 1, abort_flag)) break;
+          if (j >= 2 && !mbar_wait(&tempty[s], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t d = tmem + uint32_t(s * kTileN);
+          for (int kk = 0; kk < nk; ++kk) {
+            const int kc = kk >> 2, w = kk & 3;
+            const uint64_t ad = sdesc(su32(sA + kc * kATileBytes + w * 32));
+            const uint64_t bd = sdesc(su32(sB + (s * L.nkc + kc) * kBTileBytes + w * 32));
+            umma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          umma_commit(&tfull[s]);
+          ++issued;
+        }
+      }
+      if (*abort_flag && issued > 0) {
+        // wait (bounded) for the MMAs already issued before TMEM is freed
+        umma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never);
+      }
+    }
+  } else {
+    // ---------------- epilogue: thread = token row = TMEM lane
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const int tl = tile * kTileM + row;
+    const bool valid = tl < a.tlen;
+    const uint32_t tbase = tmem + (uint32_t(q4 * 32) << 16);
+    const int C = p.C;
+    float v[32];
+    bool ok = true;
+    // statistics of the first (up to) two tiles
+    const int nstat = ntiles < 2 ? ntiles : 2;
+    float sum = 0.f, sq = 0.f;
+    for (int j = 0; j < nstat && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&tfull[j], 0, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      for (int c = 0; c < kTileN / 32; ++c) {
+        tmem_ld32(tbase + uint32_t(j * kTileN + c * 32), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sum += v[i];
+          sq = fmaf(v[i], v[i], sq);
+        }
+      }
+    }
+    const float m = float(nstat * kTileN);
+    const float mu = sum / m;
+    const float var = fmaxf(sq / m - mu * mu, 0.f);
+    const float sd = sqrtf(var);
+    const bool keep_all = !(a.z > -1e30f);
+    const float tau = keep_all ? -INFINITY : mu + a.z * sd;
+    bool redo = !keep_all && !(sd > 0.f);
+    int cnt = 0;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int s = j & 1;
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[s], (j >> 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      for (int c = 0; c < kTileN / 32; ++c) {
+        tmem_ld32(tbase + uint32_t(s * kTileN + c * 32), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (v[i] >= tau) {
+            if (cnt < C) {
+              vals[cnt * kTileM + row] = v[i];
+              idxs[cnt * kTileM + row] = uint16_t(j * kTileN + c * 32 + i);
+            }
+            ++cnt;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[s]);
+    }
+    if (!ok) {
+      if (lane == 0) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
+    } else if (valid) {
+      const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
+      const int k = p.k;
+      if (redo || cnt < k || cnt > C) {
+        a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+      } else {
+        // exact top-k of the kept scores, sorted: bucket by value, keep the
+        // buckets that hold the k best, sort inside the multi-entry buckets
+        float vmin = INFINITY, vmax = -INFINITY;
+        for (int i = 0; i < cnt; ++i) {
+          const float x = vals[i * kTileM + row];
+          vmin = fminf(vmin, x);
+          vmax = fmaxf(vmax, x);
+        }
+        const float scale = vmax > vmin ? float(kBuckets) / (vmax - vmin) : 0.f;
+        for (int b = 0; b < kBuckets; ++b) hist[b * kTileM + row] = 0;
+        for (int i = 0; i < cnt; ++i) {
+          const int b = min(kBuckets - 1, int((vals[i * kTileM + row] - vmin) * scale));
+          hist[b * kTileM + row] += 1;
+        }
+        int bstar = kBuckets - 1, cum = 0;
+        for (int b = kBuckets - 1; b >= 0; --b) {
+          cum += hist[b * kTileM + row];
+          bstar = b;
+          if (cum >= k) break;
+        }
+        int run = 0;
+        for (int b = kBuckets - 1; b >= bstar; --b) {
+          const int hb = hist[b * kTileM + row];
+          hist[b * kTileM + row] = uint16_t(run);
+          run += hb;
+        }
+        const int nout = run;
+        uint2* out = a.surv + hr * C;
+        for (int i = 0; i < cnt; ++i) {
+          const float x = vals[i * kTileM + row];
+          const int b = min(kBuckets - 1, int((x - vmin) * scale));
+          if (b >= bstar) {
+            const int pos = hist[b * kTileM + row];
+            hist[b * kTileM + row] = uint16_t(pos + 1);
+            out[pos] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
+          }
+        }
+        int prev = 0;
+        for (int b = kBuckets - 1; b >= bstar; --b) {
+          const int end = hist[b * kTileM + row];
+          for (int i = prev + 1; i < end; ++i) {
+            const uint2 x = out[i];
+            int j2 = i - 1;
+            while (j2 >= prev && before(x, out[j2])) {
+              out[j2 + 1] = out[j2];
+              --j2;
+            }
+            out[j2 + 1] = x;
+          }
+          prev = end;
+        }
+        a.cnt[hr] = nout;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {uint32_t(kKAtom), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// z with P(N(0,1) > z) = f (bisection on the normal tail)
+double normal_upper_quantile(double f) {
+  double lo = -10.0, hi = 10.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * erfc(mid / sqrt(2.0)) > f) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+}  // namespace
+
+// Survivor capacity of a half-row: room for the expected kept count
+// (1.5 k + 16) plus a margin of 48.
+int score_tc_capacity(const sdm_dims* d) {
+  int c = (3 * d->k) / 2 + 16 + 48;
+  c = (c + 15) & ~15;
+  return c < d->n_sub ? c : d->n_sub;
+}
+
+size_t score_tc_smem(const Plan& p) { return tc_layout(p).total; }
+
+bool score_tc_supported(const sdm_dims* d) {
+  if (d->in_dtype != SDM_DTYPE_BF16) return false;
+  const int dh = d->d_qk / 2;
+  if (dh % kKAtom != 0 || dh > 256) return false;
+  if (d->n_sub % kTileN != 0 || d->n_sub > 65535) return false;
+  if ((long long)d->B * d->H * d->T >= (1LL << 31)) return false;
+  if ((long long)d->H * d->n_sub >= (1LL << 31)) return false;
+  Plan tmp;
+  tmp.dh = dh;
+  tmp.C = score_tc_capacity(d);
+  return tc_layout(tmp).total <= 227 * 1024;
+}
+
 cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const void* C1,
                             const void* C2, int t0, int tlen, int* surv_cnt, uint2* surv,
                             int* redo_rows, DevStatus* st, cudaStream_t s) {
-  (void)p; (void)q; (void)k; (void)C1; (void)C2; (void)t0; (void)tlen; (void)surv_cnt;
-  (void)surv; (void)redo_rows; (void)st; (void)s;
-  return cudaErrorNotSupported;
+  CUtensorMap mq, mk, mc1, mc2;
+  if (!encode_fn()) return cudaErrorNotSupported;
+  const uint64_t rows = uint64_t(p.BH) * p.T;
+  if (!make_map(&mq, q, rows, p.dqk, kTileM) || !make_map(&mk, k, rows, p.dqk, kTileM) ||
+      !make_map(&mc1, C1, uint64_t(p.H) * p.n, p.dh, kTileN) ||
+      !make_map(&mc2, C2, uint64_t(p.H) * p.n, p.dh, kTileN))
+    return cudaErrorInvalidValue;
+  TcArgs a;
+  a.p = p;
+  a.t0 = t0;
+  a.tlen = tlen;
+  const double f = (1.5 * p.k + 16.0) / double(p.n);
+  a.z = (f >= 1.0 || p.C >= p.n) ? -INFINITY : float(normal_upper_quantile(f));
+  a.surv = surv;
+  a.cnt = surv_cnt;
+  a.redo = redo_rows;
+  a.st = st;
+  const size_t smem = score_tc_smem(p);
+  cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((tlen + kTileM - 1) / kTileM, p.BH, 4);
+  k_score_tc<<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+  return cudaGetLastError();
 }
 
 }  // namespace sdm

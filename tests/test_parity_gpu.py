@@ -117,6 +117,22 @@ def test_forward_parity_shapes(shape):
     _check_forward(cfg, inp, ref)
 
 
+@pytest.mark.parametrize("shape", [
+    dict(T=300), dict(T=1), dict(T=129), dict(k=8, W=16, R=8), dict(W=64, R=64, k=64, T=257),
+    dict(n_sub=512, T=200), dict(B=3, H=1, T=140),
+])
+def test_tensor_core_scoring_shapes(shape):
+    """bf16 shapes served by the tcgen05 scoring kernel: ragged 128-token tiles,
+    several codebook tiles, small and large k."""
+    import sparse_memory_linear_scoring_b200 as s
+    base = config(1).with_(B=1, H=2, T=300, n_sub=256, k=32, W=64, R=64, m0_sd=0.5)
+    cfg = base.with_(**shape)
+    assert s.query_plan(s.make_dims(**cfg.dims()))["tensor_core_scoring"] == 1
+    inp = gen_inputs(cfg)
+    ref = oracle_full(inp, cfg, lists=True)
+    _check_forward(cfg, inp, ref)
+
+
 def test_fp32_wide_rows():
     cfg = config(0).with_(B=2, H=3, T=200, d_v=128, d_qk=24, n_sub=16, k=6, W=20, R=12,
                           m0_sd=1.0)
