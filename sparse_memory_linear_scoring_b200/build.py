@@ -28,17 +28,19 @@ def _stale() -> bool:
     return any(os.path.getmtime(f) > t for f in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/*.cu into libsdm.so (skipped when up to date)."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out: str = None, defines=()) -> str:
+    """Compile csrc/*.cu into libsdm.so (skipped when up to date).  `out` and
+    `defines` (e.g. "SDM_RECUR_THREADS=512") build a variant elsewhere."""
+    so = out or SO
+    if out is None and not defines and not force and not _stale():
         return SO
-    objdir = os.path.join(HERE, "_build")
+    objdir = os.path.join(os.path.dirname(so) if out else HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     procs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
-        cmd = [NVCC] + FLAGS + ["-c", src, "-o", obj]
+        cmd = [NVCC] + FLAGS + ["-D" + d for d in defines] + ["-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
@@ -52,11 +54,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed = True
     if failed:
         raise RuntimeError("nvcc failed")
-    tmp = SO + ".tmp%d" % os.getpid()
+    tmp = so + ".tmp%d" % os.getpid()
     subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp]
                           + objs + ["-lcudart"])
-    os.replace(tmp, SO)
-    return SO
+    os.replace(tmp, so)
+    return so
 
 
 if __name__ == "__main__":

@@ -17,9 +17,10 @@
 //
 // Plan (one CTA per (head, block of P steps)): the block's W+R entries per step
 // are grouped for the recurrence kernel.  Each slot belongs to one of G parts
-// (a hash of the slot); records are laid out part by part: first the slots
-// used once in the block, then the slots used several times, grouped by slot
-// in time order (write before read within a step).  A record is
+// (a hash of the slot); records are laid out part by part: the writes of slots
+// used once in the block, the reads of slots used once, then the slots used
+// several times, grouped by slot in time order (write before read within a
+// step).  A record is
 //   int4 {slot, (step_in_block << 1) | is_read, weight bits, chain length},
 // chain length = number of records of that slot in the block on its first
 // record, 0 on the others.
@@ -47,17 +48,18 @@ __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15)
 __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   MergeLayout L;
   L.Sk = p2(p.k);
+  L.Sc = ((p.ncW > p.ncR ? p.ncW : p.ncR) + 31) & ~31;
   L.Ss = p2(p.W > p.R ? p.W : p.R);
-  L.Sc = p2(p.ncW > p.ncR ? p.ncW : p.ncR);
+  if (L.Ss < L.Sc) L.Ss = L.Sc;
   L.HS = p2(2 * p.E);
   L.warps = warps;
   size_t o = 0;
   L.ent_slot = o; o = al16(o + size_t(p.E) * 4);
   L.ent_w = o; o = al16(o + size_t(p.E) * 4);
   L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR) * 4);
-  L.misc = o; o = al16(o + size_t(5 * (kMaxParts + 1) + 8) * 4);
+  L.misc = o; o = al16(o + size_t(8 * (kMaxParts + 1) + 8) * 4);
   L.uni = o;
-  L.per_warp = size_t(2 * L.Sk + L.Sc + L.Ss + 32) * 8;
+  L.per_warp = size_t(2 * L.Sk + 2 * L.Sc + L.Ss) * 8;
   L.phase2 = al16(size_t(L.HS) * 4) + al16(size_t(L.HS)) + al16(size_t(p2(p.E)) * 2);
   const size_t ph1 = L.per_warp * warps;
   o += (ph1 > L.phase2 ? ph1 : L.phase2);
@@ -134,74 +136,55 @@ __device__ __forceinline__ uint64_t warp_sort32_desc(uint64_t x) {
   return x;
 }
 
-// The r-th largest (1-based) of the nc distinct, nonzero keys in cand[]:
-// quickselect with pseudo-random pivots over the shrinking interval (L, U],
-// finished by a 32-key sort.  tmp holds 32 keys.
-__device__ uint64_t warp_select(const uint64_t* cand, int nc, int r, uint64_t* tmp) {
+// The r-th largest (1-based) of the n distinct, nonzero keys in cand[]
+// (left intact): quickselect with median-of-3 pivots; each round splits the
+// live keys around the pivot into a scratch buffer (A and B alternate, each
+// of capacity >= n) and keeps the side holding the answer; at <= 32 keys a
+// warp sort finishes.
+__device__ uint64_t warp_select(const uint64_t* cand, int n, int r, uint64_t* A, uint64_t* B) {
   const int lane = threadIdx.x & 31;
-  uint64_t L = 0, U = ~uint64_t(0);
-  int above = 0;  // keys > U
-  uint32_t seed = 0x9e3779b9u;
+  const unsigned lt_mask = lanemask_lt();
+  const uint64_t* src = cand;
+  uint64_t* bufs[2] = {A, B};
+  int which = 0;
   for (int iter = 0; iter < 4096; ++iter) {
-    int act = 0;
-    for (int i = lane; i < nc; i += 32) {
-      const uint64_t x = cand[i];
-      act += (x > L) & (x <= U);
-    }
-    int incl = act;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int tot = __shfl_sync(0xffffffffu, incl, 31);
-    if (tot <= 32) {
-      int base = 0;
-      for (int i0 = 0; i0 < nc; i0 += 32) {
-        const int i = i0 + lane;
-        const uint64_t x = i < nc ? cand[i] : 0;
-        const bool a = (i < nc) && (x > L) && (x <= U);
-        const unsigned m = __ballot_sync(0xffffffffu, a);
-        if (a) tmp[base + __popc(m & lanemask_lt())] = x;
-        base += __popc(m);
-      }
+    if (n <= 32) {
+      uint64_t x = lane < n ? src[lane] : 0;
       __syncwarp();
-      uint64_t mine = lane < tot ? tmp[lane] : 0;
-      __syncwarp();
-      mine = warp_sort32_desc(mine);
-      return __shfl_sync(0xffffffffu, mine, r - above - 1);
+      x = warp_sort32_desc(x);
+      return __shfl_sync(0xffffffffu, x, r - 1);
     }
-    seed = seed * 1664525u + 1013904223u;
-    const int j = int((uint64_t(seed >> 8) * uint64_t(tot)) >> 24);  // [0, tot)
-    const int owner = __ffs(__ballot_sync(0xffffffffu, incl > j)) - 1;
-    uint64_t piv = 0;
-    if (lane == owner) {
-      int want = j - (incl - act);
-      for (int i = lane; i < nc; i += 32) {
-        const uint64_t x = cand[i];
-        if ((x > L) && (x <= U)) {
-          if (want == 0) { piv = x; break; }
-          --want;
-        }
-      }
+    const uint64_t a = src[0], b = src[n >> 1], c = src[n - 1];
+    const uint64_t lo = a < b ? a : b, hi = a < b ? b : a;
+    const uint64_t piv = c < lo ? lo : (c > hi ? hi : c);
+    uint64_t* dst = bufs[which];
+    int front = 0, back = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const uint64_t x = i < n ? src[i] : 0;
+      const bool gt = (i < n) && x > piv;
+      const bool ls = (i < n) && x < piv;
+      const unsigned mg = __ballot_sync(0xffffffffu, gt);
+      const unsigned ml = __ballot_sync(0xffffffffu, ls);
+      if (gt) dst[front + __popc(mg & lt_mask)] = x;
+      if (ls) dst[n - 1 - (back + __popc(ml & lt_mask))] = x;
+      front += __popc(mg);
+      back += __popc(ml);
     }
-    piv = __shfl_sync(0xffffffffu, piv, owner);
-    int ge = 0;
-    for (int i = lane; i < nc; i += 32) {
-      const uint64_t x = cand[i];
-      ge += (x >= piv) & (x <= U);
-    }
-    ge = __reduce_add_sync(0xffffffffu, ge);
-    const int G = above + ge;
-    if (G == r) return piv;
-    if (G > r) {
-      L = piv;
+    __syncwarp();
+    const int ge = front + 1;
+    if (ge == r) return piv;
+    if (ge > r) {
+      src = dst;
+      n = front;
     } else {
-      U = piv - 1;
-      above = G;
+      src = dst + (n - back);
+      n = back;
+      r -= ge;
     }
+    which ^= 1;
   }
-  return 0;  // not reached: every iteration removes the pivot from (L, U]
+  return 0;  // not reached: each round removes at least the pivot
 }
 
 // Merge of one (step, side): sorted half lists (first k entries of each
@@ -209,8 +192,8 @@ __device__ uint64_t warp_select(const uint64_t* cand, int nc, int r, uint64_t* t
 // Selection order is unspecified unless `sorted` is set (then rank order).
 __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
                           int n_sel, const uint32_t* stair, int nc, const uint32_t* front, int nf,
-                          uint64_t* h1, uint64_t* h2, uint64_t* cand, uint64_t* sel,
-                          uint64_t* tmp, bool sorted, float* w_out, uint32_t* slot_out,
+                          uint64_t* h1, uint64_t* h2, uint64_t* cand, uint64_t* alt,
+                          uint64_t* sel, bool sorted, float* w_out, uint32_t* slot_out,
                           DevStatus* st, int info) {
   const int lane = threadIdx.x & 31;
   if (c1 < p.k || c1 > p.C || c2 < p.k || c2 > p.C) {
@@ -233,7 +216,7 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
     cand[i] = make_key(v, key_idx(h1[a]) * n + key_idx(h2[b]));
   }
   __syncwarp();
-  const uint64_t kth = warp_select(cand, nc, n_sel, tmp);
+  const uint64_t kth = warp_select(cand, nc, n_sel, alt, sel);
   // every candidate outside the staircase must score strictly below the kth
   const uint32_t tau = uint32_t(kth >> 32);
   bool bad = false;
@@ -244,8 +227,7 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
   }
   bool is_sorted = false;
   if (__any_sync(0xffffffffu, bad)) {
-    merge_full(h1, h2, p.k, p.n, n_sel, cand);
-    for (int i = lane; i < n_sel; i += 32) sel[i] = cand[i];
+    merge_full(h1, h2, p.k, p.n, n_sel, sel);
     is_sorted = true;
   } else {
     int base = 0;
@@ -290,12 +272,14 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   uint32_t* frontW = stairW + p.ncW;
   uint32_t* stairR = frontW + p.nfW;
   uint32_t* frontR = stairR + p.ncR;
-  int* cnt_s = reinterpret_cast<int*>(smem + L.misc);
-  int* cnt_m = cnt_s + (kMaxParts + 1);
+  int* cnt_w = reinterpret_cast<int*>(smem + L.misc);  // single-use writes per part
+  int* cnt_r = cnt_w + (kMaxParts + 1);                  // single-use reads per part
+  int* cnt_m = cnt_r + (kMaxParts + 1);                  // multi-use entries per part
   int* base = cnt_m + (kMaxParts + 1);
   int* mbase = base + (kMaxParts + 1);
-  int* fill = mbase + (kMaxParts + 1);
-  int* misc = fill + (kMaxParts + 1);  // [0] n_multi
+  int* fill_w = mbase + (kMaxParts + 1);
+  int* fill_r = fill_w + (kMaxParts + 1);
+  int* misc = fill_r + (kMaxParts + 1);  // [0] n_multi
   unsigned char* uni = smem + L.uni;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -331,8 +315,8 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
       uint64_t* h1 = reinterpret_cast<uint64_t*>(uni + L.per_warp * warp);
       uint64_t* h2 = h1 + L.Sk;
       uint64_t* cand = h2 + L.Sk;
-      uint64_t* sel = cand + L.Sc;
-      uint64_t* tmp = sel + L.Ss;
+      uint64_t* alt = cand + L.Sc;
+      uint64_t* sel = alt + L.Sc;
       for (int pi = warp; pi < 2 * np; pi += p.merge_warps) {
         const int tl = pi >> 1, side = pi & 1;
         const int tc = s0 + tl;                       // step within the chunk
@@ -342,7 +326,7 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
         uint32_t* s_out = ent_slot + tl * WR + (side ? p.W : 0);
         merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
                   io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
-                  side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, sel, tmp,
+                  side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, alt, sel,
                   io.mode == 1, w_out, s_out, st, int(hr));
         if (io.mode == 1) {
           const size_t t = size_t(bh) * p.T + t0 + tc;
@@ -382,7 +366,9 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   uint16_t* mlist = reinterpret_cast<uint16_t*>(uni + al16(size_t(L.HS) * 4) + al16(size_t(L.HS)));
   const uint32_t hmask = uint32_t(L.HS - 1);
   for (int i = tid; i < L.HS; i += blockDim.x) { hkey[i] = kEmpty; hflag[i] = 0; }
-  for (int i = tid; i <= p.G; i += blockDim.x) { cnt_s[i] = 0; cnt_m[i] = 0; fill[i] = 0; }
+  for (int i = tid; i <= p.G; i += blockDim.x) {
+    cnt_w[i] = 0; cnt_r[i] = 0; cnt_m[i] = 0; fill_w[i] = 0; fill_r[i] = 0;
+  }
   if (tid == 0) misc[0] = 0;
   __syncthreads();
   for (int e = tid; e < nent; e += blockDim.x) {
@@ -406,8 +392,10 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     if (hflag[h]) {
       mlist[atomicAdd(&misc[0], 1)] = uint16_t(e);
       atomicAdd(&cnt_m[part], 1);
+    } else if ((e % WR) < p.W) {
+      atomicAdd(&cnt_w[part], 1);
     } else {
-      atomicAdd(&cnt_s[part], 1);
+      atomicAdd(&cnt_r[part], 1);
     }
   }
   __syncthreads();
@@ -417,7 +405,7 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     for (int g = 0; g < p.G; ++g) {
       base[g] = acc;
       mbase[g] = macc;
-      acc += cnt_s[g] + cnt_m[g];
+      acc += cnt_w[g] + cnt_r[g] + cnt_m[g];
       macc += cnt_m[g];
     }
     base[p.G] = acc;
@@ -459,14 +447,16 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     while (hkey[h] != s) h = (h + 1) & hmask;
     if (hflag[h]) continue;
     const int part = slot_part(s, p.G);
-    const int pos = base[part] + atomicAdd(&fill[part], 1);
+    const bool is_read = (e % WR) >= p.W;
+    const int pos = is_read ? base[part] + cnt_w[part] + atomicAdd(&fill_r[part], 1)
+                            : base[part] + atomicAdd(&fill_w[part], 1);
     rec[pos] = make_int4(int(s), meta_of(e), __float_as_int(ent_w[e]), 1);
   }
   for (int i = tid; i < n_multi; i += blockDim.x) {
     const int e = mlist[i];
     const uint32_t s = ent_slot[e];
     const int part = slot_part(s, p.G);
-    const int pos = base[part] + cnt_s[part] + (i - mbase[part]);
+    const int pos = base[part] + cnt_w[part] + cnt_r[part] + (i - mbase[part]);
     int len = 0;
     if (i == 0 || ent_slot[mlist[i - 1]] != s) {
       int j = i + 1;
@@ -477,14 +467,19 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     }
     rec[pos] = make_int4(int(s), meta_of(e), __float_as_int(ent_w[e]), len);
   }
-  int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (p.G + 1);
-  for (int g = tid; g <= p.G; g += blockDim.x) roff[g] = base[g];
-  // the recurrence accumulates o with atomics when a head has several parts
-  if (p.G > 1) {
-    float4* o4 = reinterpret_cast<float4*>(io.o + (size_t(bh) * p.T + t0 + s0) * p.dv);
-    const int n4 = np * p.dv / 4;
-    for (int i = tid; i < n4; i += blockDim.x) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // per part g: single writes [3g, 3g+1), single reads [3g+1, 3g+2), multi-use
+  // chains [3g+2, 3g+3); entry 3G = end
+  int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (3 * p.G + 1);
+  for (int g = tid; g < p.G; g += blockDim.x) {
+    roff[3 * g] = base[g];
+    roff[3 * g + 1] = base[g] + cnt_w[g];
+    roff[3 * g + 2] = base[g] + cnt_w[g] + cnt_r[g];
   }
+  if (tid == 0) roff[3 * p.G] = base[p.G];
+  // the recurrence adds every read into o with reductions: start from zero
+  float4* o4 = reinterpret_cast<float4*>(io.o + (size_t(bh) * p.T + t0 + s0) * p.dv);
+  const int n4 = np * p.dv / 4;
+  for (int i = tid; i < n4; i += blockDim.x) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 cudaError_t launch_merge_plan(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,

@@ -73,6 +73,12 @@ __host__ __device__ inline TcLayout tc_layout(const Plan& p) {
   return L;
 }
 
+// Entries per row of the sorted-output staging area, which reuses the token
+// tile and codebook ring once every MMA has completed.
+__host__ __device__ inline int out_capacity(const TcLayout& L) {
+  return int((L.vals - L.a) / (kTileM * 8));
+}
+
 // ---- PTX wrappers -------------------------------------------------------------
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -332,15 +338,15 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       }
       for (int c = 0; c < kTileN / 32; ++c) {
         tmem_ld32(tbase + uint32_t(s * kTileN + c * 32), v);
+        const int col0 = j * kTileN + c * 32;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          if (v[i] >= tau) {
-            if (cnt < C) {
-              vals[cnt * kTileM + row] = v[i];
-              idxs[cnt * kTileM + row] = uint16_t(j * kTileN + c * 32 + i);
-            }
-            ++cnt;
+          const bool keep = v[i] >= tau;
+          if (keep && cnt < C) {
+            vals[cnt * kTileM + row] = v[i];
+            idxs[cnt * kTileM + row] = uint16_t(col0 + i);
           }
+          cnt += keep ? 1 : 0;
         }
       }
       tc_fence_before();
@@ -351,6 +357,7 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
     } else if (valid) {
       const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
       const int k = p.k;
+      bool continue_out = true;
       if (redo || cnt < k || cnt > C) {
         a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
       } else {
@@ -381,31 +388,47 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
           run += hb;
         }
         const int nout = run;
-        uint2* out = a.surv + hr * C;
-        for (int i = 0; i < cnt; ++i) {
+        const int ocap = out_capacity(L);
+        if (nout > ocap) {
+          a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+          continue_out = false;
+        }
+        // every MMA has completed (the last tfull wait), so the token tile and
+        // codebook ring are free: stage the sorted list there, column = row
+        uint2* out = reinterpret_cast<uint2*>(smem + L.a);
+        for (int i = 0; i < cnt && continue_out; ++i) {
           const float x = vals[i * kTileM + row];
           const int b = min(kBuckets - 1, int((x - vmin) * scale));
           if (b >= bstar) {
             const int pos = hist[b * kTileM + row];
             hist[b * kTileM + row] = uint16_t(pos + 1);
-            out[pos] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
+            out[pos * kTileM + row] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
           }
         }
-        int prev = 0;
-        for (int b = kBuckets - 1; b >= bstar; --b) {
-          const int end = hist[b * kTileM + row];
-          for (int i = prev + 1; i < end; ++i) {
-            const uint2 x = out[i];
-            int j2 = i - 1;
-            while (j2 >= prev && before(x, out[j2])) {
-              out[j2 + 1] = out[j2];
-              --j2;
+        if (continue_out) {
+          int prev = 0;
+          for (int b = kBuckets - 1; b >= bstar; --b) {
+            const int end = hist[b * kTileM + row];
+            for (int i = prev + 1; i < end; ++i) {
+              const uint2 x = out[i * kTileM + row];
+              int j2 = i - 1;
+              while (j2 >= prev && before(x, out[j2 * kTileM + row])) {
+                out[(j2 + 1) * kTileM + row] = out[j2 * kTileM + row];
+                --j2;
+              }
+              out[(j2 + 1) * kTileM + row] = x;
             }
-            out[j2 + 1] = x;
+            prev = end;
           }
-          prev = end;
+          uint4* g = reinterpret_cast<uint4*>(a.surv + hr * C);
+          int i = 0;
+          for (; i + 1 < nout; i += 2) {
+            const uint2 x0 = out[i * kTileM + row], x1 = out[(i + 1) * kTileM + row];
+            g[i >> 1] = make_uint4(x0.x, x0.y, x1.x, x1.y);
+          }
+          if (i < nout) a.surv[hr * C + i] = out[i * kTileM + row];
+          a.cnt[hr] = nout;
         }
-        a.cnt[hr] = nout;
       }
     }
   }
@@ -475,7 +498,8 @@ bool score_tc_supported(const sdm_dims* d) {
   Plan tmp;
   tmp.dh = dh;
   tmp.C = score_tc_capacity(d);
-  return tc_layout(tmp).total <= 227 * 1024;
+  const TcLayout L = tc_layout(tmp);
+  return L.total <= 227 * 1024 && out_capacity(L) >= d->k + 16;
 }
 
 cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const void* C1,

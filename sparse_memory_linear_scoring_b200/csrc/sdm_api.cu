@@ -73,6 +73,10 @@ int make_plan(const sdm_dims* d, Plan* p) {
   if (p->ncW < p->W || p->ncR < p->R) return SDM_ERR_UNSUPPORTED;
   int P = kMaxBlockEntries / (p->W + p->R);
   if (P > 1024) P = 1024;
+  // the recurrence stages v (double-buffered) and an fp32 accumulator per step
+  const int vbytes = p->dtype == SDM_DTYPE_F32 ? 4 : 2;
+  const int p_smem = int((96 * 1024) / (p->dv * (2 * vbytes + 4)));
+  if (P > p_smem) P = p_smem;
   if (p->T > 0 && P > p->T) P = p->T;
   if (P < 1) P = 1;
   p->P = P;
@@ -84,7 +88,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
   // time chunk: bounded workspace
   const size_t per_step = size_t(p->BH) * (4 * 4 + size_t(4) * p->C * 8 + 4 * 4 +
                                            size_t(p->W + p->R) * 16) +
-                          (size_t(p->BH) * (p->G + 1) * 4 + size_t(P) - 1) / size_t(P);
+                          (size_t(p->BH) * (3 * p->G + 1) * 4 + size_t(P) - 1) / size_t(P);
   const long long Tround = ((long long)(p->T > 0 ? p->T : 1) + P - 1) / P * P;
   long long Tc = (long long)(kChunkBudget / per_step) / P * P;
   if (Tc < P) Tc = P;
@@ -107,7 +111,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
   p->off_surv = o; o = align256(o + nhr * p->C * 8);
   p->off_redo = o; o = align256(o + nhr * 4);
   p->off_rec = o; o = align256(o + size_t(p->BH) * p->nblk * p->E * 16);
-  p->off_roff = o; o = align256(o + size_t(p->BH) * p->nblk * (p->G + 1) * 4);
+  p->off_roff = o; o = align256(o + size_t(p->BH) * p->nblk * (3 * p->G + 1) * 4);
   p->total = o;
   return SDM_OK;
 }

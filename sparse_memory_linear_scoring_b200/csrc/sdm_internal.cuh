@@ -18,12 +18,22 @@ namespace sdm {
 
 // Fixed launch targets (depend on nothing but the problem sizes, so the
 // workspace size is a function of the dims alone).
-constexpr int kTargetCtas = 296;        // 2 x 148 SMs of a B200
+#ifndef SDM_TARGET_CTAS
+#define SDM_TARGET_CTAS 296
+#endif
+#ifndef SDM_RECUR_THREADS
+#define SDM_RECUR_THREADS 256
+#endif
+#ifndef SDM_RECUR_UNROLL
+#define SDM_RECUR_UNROLL 8
+#endif
+constexpr int kTargetCtas = SDM_TARGET_CTAS;  // recurrence CTAs aimed for (2 x 148 SMs)
 constexpr int kMaxParts = 64;           // slot parts per head in the recurrence
 constexpr int kMaxBlockEntries = 8192;  // list entries per (head, block) in a plan
 constexpr size_t kChunkBudget = size_t(1) << 30;  // workspace bytes per time chunk
-constexpr int kMergeThreads = 256;
-constexpr int kRecurThreads = 256;
+constexpr int kMergeThreads = 512;
+constexpr int kRecurThreads = SDM_RECUR_THREADS;
+constexpr int kRecurUnroll = SDM_RECUR_UNROLL;
 
 // Everything the kernels need to know about one call.
 struct Plan {
