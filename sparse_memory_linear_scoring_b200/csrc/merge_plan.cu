@@ -15,6 +15,9 @@
 // bmax(a)), since sums fall along each row; if the frontier check fails, an
 // exact search over all k x k candidates runs instead.
 //
+// The merge kernel writes the lists (slot, weight) of every step; the plan
+// kernel reads them back (or a caller's lists) and builds the recurrence plan.
+//
 // Plan (one CTA per (head, block of P steps)): the block's W+R entries per step
 // are grouped for the recurrence kernel.  Each slot belongs to one of G parts
 // (a hash of the slot); records are laid out part by part: the writes of slots
@@ -31,12 +34,6 @@ namespace sdm {
 constexpr uint32_t kEmpty = 0xffffffffu;
 constexpr uint32_t kInvalid = 0xffffffffu;
 
-struct MergeLayout {
-  size_t ent_slot, ent_w, stair, misc, uni, total;
-  int Sk, Sc, Ss, HS, warps;
-  size_t per_warp, phase2;
-};
-
 __host__ __device__ inline int p2(int x) {
   int p = 2;
   while (p < x) p <<= 1;
@@ -45,29 +42,57 @@ __host__ __device__ inline int p2(int x) {
 
 __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
 
+// k_merge: staircase tables, then per warp: two sorted half lists (h1, h2),
+// the candidate scores and two select buffers (32-bit), and the selection.
+struct MergeLayout {
+  size_t stair, uni, total, per_warp;
+  int Sk, Sc, Ss, warps;
+};
+
 __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   MergeLayout L;
   L.Sk = p2(p.k);
   L.Sc = ((p.ncW > p.ncR ? p.ncW : p.ncR) + 31) & ~31;
   L.Ss = p2(p.W > p.R ? p.W : p.R);
   if (L.Ss < L.Sc) L.Ss = L.Sc;
-  L.HS = p2(2 * p.E);
   L.warps = warps;
   size_t o = 0;
-  L.ent_slot = o; o = al16(o + size_t(p.E) * 4);
-  L.ent_w = o; o = al16(o + size_t(p.E) * 4);
   L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR) * 4);
-  L.misc = o; o = al16(o + size_t(8 * (kMaxParts + 1) + 8) * 4);
   L.uni = o;
-  L.per_warp = size_t(2 * L.Sk + 2 * L.Sc + L.Ss) * 8;
-  L.phase2 = al16(size_t(L.HS) * 4) + al16(size_t(L.HS)) + al16(size_t(p2(p.E)) * 2);
-  const size_t ph1 = L.per_warp * warps;
-  o += (ph1 > L.phase2 ? ph1 : L.phase2);
+  L.per_warp = size_t(2 * L.Sk + L.Ss) * 8 + size_t(3 * L.Sc) * 4;
+  o += L.per_warp * warps;
   L.total = al16(o);
   return L;
 }
 
 size_t merge_smem_bytes(const Plan& p, int warps) { return merge_layout(p, warps).total; }
+
+// k_plan: the block's entries, a hash table of its slots (bit 31 marks a slot
+// used more than once), the multi-use list, and per-warp class counters.
+struct PlanLayout {
+  size_t ent_slot, ent_w, ent_key, hkey, mlist, cnt, off, misc, total;
+  int HS;
+};
+
+__host__ __device__ inline PlanLayout plan_layout(const Plan& p) {
+  PlanLayout L;
+  L.HS = p2(2 * p.E);
+  const int nk = 3 * p.G;
+  const int nw = kMergeThreads / 32;
+  size_t o = 0;
+  L.ent_slot = o; o = al16(o + size_t(p.E) * 4);
+  L.ent_w = o; o = al16(o + size_t(p.E) * 4);
+  L.ent_key = o; o = al16(o + size_t(p.E));
+  L.hkey = o; o = al16(o + size_t(L.HS) * 4);
+  L.mlist = o; o = al16(o + size_t(p2(p.E)) * 2);
+  L.cnt = o; o = al16(o + size_t(nw) * nk * 4);
+  L.off = o; o = al16(o + size_t(nw) * nk * 4);
+  L.misc = o; o = al16(o + size_t(2 * nk + 2 * kMaxParts + 8) * 4);
+  L.total = o;
+  return L;
+}
+
+size_t plan_smem_bytes(const Plan& p) { return plan_layout(p).total; }
 
 // ------------------------------------------------------------------ merge (warp)
 // Exact top-n_sel of all k*k candidates by a bitwise search over the 64-bit
@@ -136,32 +161,64 @@ __device__ __forceinline__ uint64_t warp_sort32_desc(uint64_t x) {
   return x;
 }
 
-// The r-th largest (1-based) of the n distinct, nonzero keys in cand[]
-// (left intact): quickselect with median-of-3 pivots; each round splits the
-// live keys around the pivot into a scratch buffer (A and B alternate, each
-// of capacity >= n) and keeps the side holding the answer; at <= 32 keys a
-// warp sort finishes.
-__device__ uint64_t warp_select(const uint64_t* cand, int n, int r, uint64_t* A, uint64_t* B) {
+// Descending bitonic sort of one 32-bit key per lane across the warp.
+__device__ __forceinline__ uint32_t warp_sort32_desc_u32(uint32_t x) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, x, stride);
+      const bool desc = (lane & size) == 0 || size == 32;
+      const bool lower = (lane & stride) == 0;
+      x = (lower == desc) ? max(x, y) : min(x, y);
+    }
+  }
+  return x;
+}
+
+// Ascending bitonic sort of S (power of two) 32-bit keys in shared memory by
+// one warp.
+__device__ void warp_sort_asc_u32(uint32_t* a, int S) {
+  const int lane = threadIdx.x & 31;
+  for (int size = 2; size <= S; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = lane; i < (S >> 1); i += 32) {
+        const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
+        const int hi = lo + stride;
+        const uint32_t x = a[lo], y = a[hi];
+        const bool asc = (lo & size) == 0;
+        if (asc ? (x > y) : (x < y)) { a[lo] = y; a[hi] = x; }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// The r-th largest (1-based, counting repeats) of the n values in cand[]
+// (left intact): quickselect with median-of-3 pivots and a three-way split;
+// each round moves the values above / below the pivot into a scratch buffer
+// (A and B alternate, each of capacity >= n); at <= 32 values a warp sort
+// finishes.
+__device__ uint32_t warp_select32(const uint32_t* cand, int n, int r, uint32_t* A, uint32_t* B) {
   const int lane = threadIdx.x & 31;
   const unsigned lt_mask = lanemask_lt();
-  const uint64_t* src = cand;
-  uint64_t* bufs[2] = {A, B};
+  const uint32_t* src = cand;
   int which = 0;
   for (int iter = 0; iter < 4096; ++iter) {
     if (n <= 32) {
-      uint64_t x = lane < n ? src[lane] : 0;
+      uint32_t x = lane < n ? src[lane] : 0u;
       __syncwarp();
-      x = warp_sort32_desc(x);
+      x = warp_sort32_desc_u32(x);
       return __shfl_sync(0xffffffffu, x, r - 1);
     }
-    const uint64_t a = src[0], b = src[n >> 1], c = src[n - 1];
-    const uint64_t lo = a < b ? a : b, hi = a < b ? b : a;
-    const uint64_t piv = c < lo ? lo : (c > hi ? hi : c);
-    uint64_t* dst = bufs[which];
+    const uint32_t a = src[0], b = src[n >> 1], c = src[n - 1];
+    const uint32_t piv = max(min(a, b), min(max(a, b), c));
+    uint32_t* dst = which ? B : A;
     int front = 0, back = 0;
     for (int i0 = 0; i0 < n; i0 += 32) {
       const int i = i0 + lane;
-      const uint64_t x = i < n ? src[i] : 0;
+      const uint32_t x = i < n ? src[i] : 0u;
       const bool gt = (i < n) && x > piv;
       const bool ls = (i < n) && x < piv;
       const unsigned mg = __ballot_sync(0xffffffffu, gt);
@@ -172,19 +229,20 @@ __device__ uint64_t warp_select(const uint64_t* cand, int n, int r, uint64_t* A,
       back += __popc(ml);
     }
     __syncwarp();
-    const int ge = front + 1;
-    if (ge == r) return piv;
-    if (ge > r) {
+    const int eq = n - front - back;
+    if (r <= front) {
       src = dst;
       n = front;
+    } else if (r <= front + eq) {
+      return piv;
     } else {
       src = dst + (n - back);
       n = back;
-      r -= ge;
+      r -= front + eq;
     }
     which ^= 1;
   }
-  return 0;  // not reached: each round removes at least the pivot
+  return 0u;  // not reached: each round removes at least the pivot's value
 }
 
 // Merge of one (step, side): sorted half lists (first k entries of each
@@ -192,7 +250,7 @@ __device__ uint64_t warp_select(const uint64_t* cand, int n, int r, uint64_t* A,
 // Selection order is unspecified unless `sorted` is set (then rank order).
 __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
                           int n_sel, const uint32_t* stair, int nc, const uint32_t* front, int nf,
-                          uint64_t* h1, uint64_t* h2, uint64_t* cand, uint64_t* alt,
+                          uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* alt,
                           uint64_t* sel, bool sorted, float* w_out, uint32_t* slot_out,
                           DevStatus* st, int info) {
   const int lane = threadIdx.x & 31;
@@ -209,34 +267,89 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
   }
   __syncwarp();
   const uint32_t n = uint32_t(p.n);
+  // staircase candidate scores (ordered 32-bit images of the float32 sums)
   for (int i = lane; i < nc; i += 32) {
     const uint32_t ab = stair[i];
-    const int a = ab & 0xffff, b = ab >> 16;
-    const float v = key_val(h1[a]) + key_val(h2[b]);
-    cand[i] = make_key(v, key_idx(h1[a]) * n + key_idx(h2[b]));
+    cand[i] = f2ord(key_val(h1[ab & 0xffff]) + key_val(h2[ab >> 16]));
   }
   __syncwarp();
-  const uint64_t kth = warp_select(cand, nc, n_sel, alt, sel);
-  // every candidate outside the staircase must score strictly below the kth
-  const uint32_t tau = uint32_t(kth >> 32);
+  const uint32_t vstar = warp_select32(cand, nc, n_sel, alt, alt + (nc + 31) / 32 * 32);
+  // exact when every candidate outside the staircase scores strictly below the
+  // n_sel-th and no other candidate ties it
+  int n_gt = 0, n_eq = 0;
+  for (int i = lane; i < nc; i += 32) {
+    const uint32_t x = cand[i];
+    n_gt += x > vstar;
+    n_eq += x == vstar;
+  }
+  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
   bool bad = false;
   for (int i = lane; i < nf; i += 32) {
     const uint32_t ab = front[i];
-    const int a = ab & 0xffff, b = ab >> 16;
-    bad |= f2ord(key_val(h1[a]) + key_val(h2[b])) >= tau;
+    bad |= f2ord(key_val(h1[ab & 0xffff]) + key_val(h2[ab >> 16])) >= vstar;
   }
   bool is_sorted = false;
-  if (__any_sync(0xffffffffu, bad)) {
-    merge_full(h1, h2, p.k, p.n, n_sel, sel);
-    is_sorted = true;
+  if (__any_sync(0xffffffffu, bad) || n_gt + n_eq != n_sel) {
+    // Ties at vstar.  Every candidate outside the staircase is dominated by at
+    // least n_sel staircase candidates, so it scores <= vstar: the selection is
+    // the n_gt staircase candidates above vstar plus the lowest slots among all
+    // k*k candidates equal to vstar.
+    const int kk = p.k * p.k;
+    int tcap = 1;  // largest power of two that fits the scratch (2 * Sc entries)
+    while (2 * tcap <= 2 * (((p.ncW > p.ncR ? p.ncW : p.ncR) + 31) & ~31)) tcap *= 2;
+    int n_tie = 0;
+    for (int i0 = 0; i0 < kk; i0 += 32) {
+      const int i = i0 + lane;
+      bool tie = false;
+      uint32_t slot = 0;
+      if (i < kk) {
+        const int a = i / p.k, b = i - a * p.k;
+        tie = f2ord(key_val(h1[a]) + key_val(h2[b])) == vstar;
+        slot = key_idx(h1[a]) * n + key_idx(h2[b]);
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, tie);
+      const int pos = n_tie + __popc(m & lanemask_lt());
+      if (tie && pos < tcap) alt[pos] = slot;
+      n_tie += __popc(m);
+    }
+    __syncwarp();
+    if (n_tie > tcap) {
+      merge_full(h1, h2, p.k, p.n, n_sel, sel);  // pathological ties only
+      is_sorted = true;
+    } else {
+      const int S = p2(n_tie);
+      for (int i = n_tie + lane; i < S; i += 32) alt[i] = 0xffffffffu;
+      __syncwarp();
+      warp_sort_asc_u32(alt, S);
+      int base = 0;
+      for (int i0 = 0; i0 < nc; i0 += 32) {
+        const int i = i0 + lane;
+        const bool take = (i < nc) && cand[i] > vstar;
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (take) {
+          const uint32_t ab = stair[i];
+          const uint64_t a = h1[ab & 0xffff], b = h2[ab >> 16];
+          sel[base + __popc(m & lanemask_lt())] =
+              (uint64_t(cand[i]) << 32) | uint64_t(~(key_idx(a) * n + key_idx(b)));
+        }
+        base += __popc(m);
+      }
+      for (int j = lane; j < n_sel - base; j += 32)
+        sel[base + j] = (uint64_t(vstar) << 32) | uint64_t(~alt[j]);
+    }
   } else {
     int base = 0;
     for (int i0 = 0; i0 < nc; i0 += 32) {
       const int i = i0 + lane;
-      const uint64_t x = i < nc ? cand[i] : 0;
-      const bool take = (i < nc) && x >= kth;
+      const bool take = (i < nc) && cand[i] >= vstar;
       const unsigned m = __ballot_sync(0xffffffffu, take);
-      if (take) sel[base + __popc(m & lanemask_lt())] = x;
+      if (take) {
+        const uint32_t ab = stair[i];
+        const uint64_t a = h1[ab & 0xffff], b = h2[ab >> 16];
+        sel[base + __popc(m & lanemask_lt())] =
+            (uint64_t(cand[i]) << 32) | uint64_t(~(key_idx(a) * n + key_idx(b)));
+      }
       base += __popc(m);
     }
   }
@@ -261,116 +374,125 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
   __syncwarp();
 }
 
-// ------------------------------------------------------------------ kernel
-__global__ void __launch_bounds__(kMergeThreads)
-k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
+// ------------------------------------------------------------------ kernels
+// Staircase rows a < k with bm(a) = min(k, n_sel / (a+1)) columns, and the
+// frontier cell (a, bm(a)) of each row that stops short of k (rows past the
+// last non-empty one contribute only their first empty cell).  One warp.
+__device__ void build_staircase(int k, int n_sel, uint32_t* stair, uint32_t* front) {
+  const int lane = threadIdx.x & 31;
+  int obase = 0, fbase = 0, prev_last = -1;
+  for (int a0 = 0; a0 < k; a0 += 32) {
+    const int a = a0 + lane;
+    const int bm = a < k ? min(k, n_sel / (a + 1)) : 0;
+    const int prev = __shfl_up_sync(0xffffffffu, bm, 1);
+    const int pbm = lane == 0 ? prev_last : prev;
+    const bool fr = a < k && bm < k && !(bm == 0 && pbm == 0);
+    int incl = bm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned fm = __ballot_sync(0xffffffffu, fr);
+    const int start = obase + incl - bm;
+    for (int b = 0; b < bm; ++b) stair[start + b] = uint32_t(a) | (uint32_t(b) << 16);
+    if (fr) front[fbase + __popc(fm & lanemask_lt())] = uint32_t(a) | (uint32_t(bm) << 16);
+    obase += __shfl_sync(0xffffffffu, incl, 31);
+    fbase += __popc(fm);
+    prev_last = __shfl_sync(0xffffffffu, bm, 31);
+  }
+}
+
+// One CTA per (head, kMergeSteps steps); one warp per (step, side).  Writes
+// the W write and R read (slot, weight) pairs of each step to the lists
+// (row = bh * list_T + list_t0 + step), in rank order when `sorted`.
+__global__ void __launch_bounds__(kMergeWarps * 32)
+k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const MergeLayout L = merge_layout(p, p.merge_warps);
-  uint32_t* ent_slot = reinterpret_cast<uint32_t*>(smem + L.ent_slot);
-  float* ent_w = reinterpret_cast<float*>(smem + L.ent_w);
+  const MergeLayout L = merge_layout(p, kMergeWarps);
   uint32_t* stairW = reinterpret_cast<uint32_t*>(smem + L.stair);
   uint32_t* frontW = stairW + p.ncW;
   uint32_t* stairR = frontW + p.nfW;
   uint32_t* frontR = stairR + p.ncR;
-  int* cnt_w = reinterpret_cast<int*>(smem + L.misc);  // single-use writes per part
-  int* cnt_r = cnt_w + (kMaxParts + 1);                  // single-use reads per part
-  int* cnt_m = cnt_r + (kMaxParts + 1);                  // multi-use entries per part
-  int* base = cnt_m + (kMaxParts + 1);
-  int* mbase = base + (kMaxParts + 1);
-  int* fill_w = mbase + (kMaxParts + 1);
-  int* fill_r = fill_w + (kMaxParts + 1);
-  int* misc = fill_r + (kMaxParts + 1);  // [0] n_multi
-  unsigned char* uni = smem + L.uni;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int bh = blockIdx.y;
+  const int s0 = blockIdx.x * kMergeSteps;
+  if (s0 >= tlen) return;
+  const int np = min(kMergeSteps, tlen - s0);
+  if (warp == 0) build_staircase(p.k, p.W, stairW, frontW);
+  if (warp == 1) build_staircase(p.k, p.R, stairR, frontR);
+  __syncthreads();
+  unsigned char* mine = smem + L.uni + L.per_warp * warp;
+  uint64_t* h1 = reinterpret_cast<uint64_t*>(mine);
+  uint64_t* h2 = h1 + L.Sk;
+  uint64_t* sel = h2 + L.Sk;
+  uint32_t* cand = reinterpret_cast<uint32_t*>(sel + L.Ss);
+  uint32_t* alt = cand + L.Sc;
+  for (int pi = warp; pi < 2 * np; pi += kMergeWarps) {
+    const int tc = s0 + (pi >> 1), side = pi & 1;
+    const size_t hr = (size_t(bh) * p.Tc + tc) * 4 + side * 2;
+    const int n_sel = side ? p.R : p.W;
+    const size_t row = size_t(bh) * io.list_T + io.list_t0 + tc;
+    float* w_out = (side ? io.out_wr : io.out_ww) + row * n_sel;
+    uint32_t* s_out = reinterpret_cast<uint32_t*>(side ? io.out_ir : io.out_iw) + row * n_sel;
+    merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
+              io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
+              side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, alt, sel,
+              io.sorted != 0, w_out, s_out, st, int(hr));
+  }
+}
+
+// One CTA per (head, block of P steps): group the block's list entries into
+// the recurrence plan (see the file header) and zero the block's rows of o.
+__global__ void __launch_bounds__(kMergeThreads)
+k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const PlanLayout L = plan_layout(p);
+  uint32_t* ent_slot = reinterpret_cast<uint32_t*>(smem + L.ent_slot);
+  float* ent_w = reinterpret_cast<float*>(smem + L.ent_w);
+  uint8_t* ent_key = smem + L.ent_key;
+  uint32_t* hkey = reinterpret_cast<uint32_t*>(smem + L.hkey);
+  uint16_t* mlist = reinterpret_cast<uint16_t*>(smem + L.mlist);
+  const int NK = 3 * p.G;                 // class keys: part * 3 + {single write, read, multi}
+  constexpr int NW = kMergeThreads / 32;
+  int* cnt = reinterpret_cast<int*>(smem + L.cnt);   // [NW][NK]
+  int* off = reinterpret_cast<int*>(smem + L.off);   // [NW][NK]
+  int* tot = reinterpret_cast<int*>(smem + L.misc);  // [NK] totals, then [NK] bases
+  int* kbase = tot + NK;
+  int* mbase = kbase + NK;                           // [G] start of a part's multis in mlist
+  int* misc = mbase + kMaxParts;                     // [0] n_multi
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int WR = p.W + p.R;
-  const int s0 = blk * p.P;                 // first step of the block within the chunk
+  const int s0 = blk * p.P;
   if (s0 >= tlen) return;
   const int np = min(p.P, tlen - s0);
   const int nent = np * WR;
-
-  if (io.mode != 2) {
-    // staircase tables: row a holds columns b < min(k, n_sel / (a+1))
-    if (tid == 0) {
-      int oc = 0, of = 0, prev = -1;
-      for (int a = 0; a < p.k; ++a) {
-        const int bm = min(p.k, p.W / (a + 1));
-        for (int b = 0; b < bm; ++b) stairW[oc++] = uint32_t(a) | (uint32_t(b) << 16);
-        if (bm < p.k && !(bm == 0 && prev == 0)) frontW[of++] = uint32_t(a) | (uint32_t(bm) << 16);
-        prev = bm;
-      }
-    } else if (tid == 32) {
-      int oc = 0, of = 0, prev = -1;
-      for (int a = 0; a < p.k; ++a) {
-        const int bm = min(p.k, p.R / (a + 1));
-        for (int b = 0; b < bm; ++b) stairR[oc++] = uint32_t(a) | (uint32_t(b) << 16);
-        if (bm < p.k && !(bm == 0 && prev == 0)) frontR[of++] = uint32_t(a) | (uint32_t(bm) << 16);
-        prev = bm;
-      }
-    }
-    __syncthreads();
-    // ---- phase 1: merges, one warp per (step, side)
-    if (warp < p.merge_warps) {
-      uint64_t* h1 = reinterpret_cast<uint64_t*>(uni + L.per_warp * warp);
-      uint64_t* h2 = h1 + L.Sk;
-      uint64_t* cand = h2 + L.Sk;
-      uint64_t* alt = cand + L.Sc;
-      uint64_t* sel = alt + L.Sc;
-      for (int pi = warp; pi < 2 * np; pi += p.merge_warps) {
-        const int tl = pi >> 1, side = pi & 1;
-        const int tc = s0 + tl;                       // step within the chunk
-        const size_t hr = (size_t(bh) * p.Tc + tc) * 4 + side * 2;
-        const int n_sel = side ? p.R : p.W;
-        float* w_out = ent_w + tl * WR + (side ? p.W : 0);
-        uint32_t* s_out = ent_slot + tl * WR + (side ? p.W : 0);
-        merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
-                  io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
-                  side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, alt, sel,
-                  io.mode == 1, w_out, s_out, st, int(hr));
-        if (io.mode == 1) {
-          const size_t t = size_t(bh) * p.T + t0 + tc;
-          int32_t* oi = side ? io.out_ir : io.out_iw;
-          float* ow = side ? io.out_wr : io.out_ww;
-          for (int i = lane; i < n_sel; i += 32) {
-            oi[t * n_sel + i] = int32_t(s_out[i]);
-            ow[t * n_sel + i] = w_out[i];
-          }
-        }
-      }
-    }
-    if (io.mode == 1) return;
-  } else {
-    // ---- lists given: validate and copy
-    for (int e = tid; e < nent; e += blockDim.x) {
-      const int tl = e / WR, j = e - tl * WR;
-      const size_t t = size_t(bh) * p.T + t0 + s0 + tl;
-      int32_t s;
-      float w;
-      if (j < p.W) { s = io.in_iw[t * p.W + j]; w = io.in_ww[t * p.W + j]; }
-      else { s = io.in_ir[t * p.R + (j - p.W)]; w = io.in_wr[t * p.R + (j - p.W)]; }
-      if (s < 0 || (long long)s >= p.N) {
-        dev_flag(st, SDM_DEV_BAD_INDEX, int(t));
-        ent_slot[e] = kInvalid;
-      } else {
-        ent_slot[e] = uint32_t(s);
-      }
-      ent_w[e] = w;
-    }
-  }
-  __syncthreads();
-
-  // ---- phase 2: plan.  Hash table of the block's slots -> used once or more.
-  uint32_t* hkey = reinterpret_cast<uint32_t*>(uni);
-  unsigned char* hflag = uni + al16(size_t(L.HS) * 4);
-  uint16_t* mlist = reinterpret_cast<uint16_t*>(uni + al16(size_t(L.HS) * 4) + al16(size_t(L.HS)));
   const uint32_t hmask = uint32_t(L.HS - 1);
-  for (int i = tid; i < L.HS; i += blockDim.x) { hkey[i] = kEmpty; hflag[i] = 0; }
-  for (int i = tid; i <= p.G; i += blockDim.x) {
-    cnt_w[i] = 0; cnt_r[i] = 0; cnt_m[i] = 0; fill_w[i] = 0; fill_r[i] = 0;
-  }
+  constexpr uint32_t kMulti = 0x80000000u;
+
+  for (int i = tid; i < L.HS; i += blockDim.x) hkey[i] = kEmpty;
+  for (int i = tid; i < NW * NK; i += blockDim.x) cnt[i] = 0;
   if (tid == 0) misc[0] = 0;
+  // entries, in step order, writes before reads
+  for (int e = tid; e < nent; e += blockDim.x) {
+    const int tl = e / WR, j = e - tl * WR;
+    const size_t row = size_t(bh) * io.list_T + io.list_t0 + s0 + tl;
+    int32_t s;
+    float w;
+    if (j < p.W) { s = io.iw[row * p.W + j]; w = io.ww[row * p.W + j]; }
+    else { s = io.ir[row * p.R + (j - p.W)]; w = io.wr[row * p.R + (j - p.W)]; }
+    if (s < 0 || (long long)s >= p.N) {
+      if (io.validate) dev_flag(st, SDM_DEV_BAD_INDEX, int(size_t(bh) * p.T + t0 + s0 + tl));
+      ent_slot[e] = kInvalid;
+    } else {
+      ent_slot[e] = uint32_t(s);
+    }
+    ent_w[e] = w;
+  }
   __syncthreads();
+  // hash table of the block's slots; a second sighting sets bit 31
   for (int e = tid; e < nent; e += blockDim.x) {
     const uint32_t s = ent_slot[e];
     if (s == kInvalid) continue;
@@ -378,38 +500,65 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     for (;;) {
       const uint32_t old = atomicCAS(&hkey[h], kEmpty, s);
       if (old == kEmpty) break;
-      if (old == s) { hflag[h] = 1; break; }
+      if ((old & ~kMulti) == s) {
+        if (!(old & kMulti)) atomicOr(&hkey[h], kMulti);
+        break;
+      }
       h = (h + 1) & hmask;
     }
   }
   __syncthreads();
-  for (int e = tid; e < nent; e += blockDim.x) {
+  // classify; count per (warp, key).  Warp w takes entries [w*chunk, (w+1)*chunk).
+  const int chunk = (nent + NW - 1) / NW;
+  const int e_lo = warp * chunk, e_hi = min(nent, e_lo + chunk);
+  for (int e = e_lo + lane; e < e_hi; e += 32) {
     const uint32_t s = ent_slot[e];
-    if (s == kInvalid) continue;
-    uint32_t h = mix32(s) & hmask;
-    while (hkey[h] != s) h = (h + 1) & hmask;
-    const int part = slot_part(s, p.G);
-    if (hflag[h]) {
-      mlist[atomicAdd(&misc[0], 1)] = uint16_t(e);
-      atomicAdd(&cnt_m[part], 1);
-    } else if ((e % WR) < p.W) {
-      atomicAdd(&cnt_w[part], 1);
-    } else {
-      atomicAdd(&cnt_r[part], 1);
+    uint8_t key = 0xff;
+    if (s != kInvalid) {
+      uint32_t h = mix32(s) & hmask;
+      while ((hkey[h] & ~kMulti) != s) h = (h + 1) & hmask;
+      const int part = slot_part(s, p.G);
+      int cls;
+      if (hkey[h] & kMulti) {
+        cls = 2;
+        mlist[atomicAdd(&misc[0], 1)] = uint16_t(e);
+      } else {
+        cls = (e % WR) < p.W ? 0 : 1;
+      }
+      key = uint8_t(part * 3 + cls);
+      atomicAdd(&cnt[warp * NK + key], 1);
     }
+    ent_key[e] = key;
   }
   __syncthreads();
-  const int n_multi = misc[0];
+  // totals per key, bases in part-major key order, per-warp offsets
+  for (int kk = tid; kk < NK; kk += blockDim.x) {
+    int t = 0;
+    for (int w = 0; w < NW; ++w) t += cnt[w * NK + kk];
+    tot[kk] = t;
+  }
+  __syncthreads();
   if (tid == 0) {
     int acc = 0, macc = 0;
-    for (int g = 0; g < p.G; ++g) {
-      base[g] = acc;
-      mbase[g] = macc;
-      acc += cnt_w[g] + cnt_r[g] + cnt_m[g];
-      macc += cnt_m[g];
+    for (int kk = 0; kk < NK; ++kk) {
+      kbase[kk] = acc;
+      acc += tot[kk];
+      if (kk % 3 == 2) {
+        mbase[kk / 3] = macc;
+        macc += tot[kk];
+      }
     }
-    base[p.G] = acc;
+    misc[1] = acc;
   }
+  __syncthreads();
+  for (int kk = tid; kk < NK; kk += blockDim.x) {
+    int run = kbase[kk];
+    for (int w = 0; w < NW; ++w) {
+      off[w * NK + kk] = run;
+      run += cnt[w * NK + kk];
+    }
+  }
+  const int n_multi = misc[0];
   // sort the multi-use entries by (part, slot, entry) -- ascending bitonic
   {
     const int S = n_multi > 1 ? p2(n_multi) : 1;
@@ -440,23 +589,19 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     const int tl = e / WR;
     return (tl << 1) | ((e - tl * WR) >= p.W ? 1 : 0);
   };
-  for (int e = tid; e < nent; e += blockDim.x) {
-    const uint32_t s = ent_slot[e];
-    if (s == kInvalid) continue;
-    uint32_t h = mix32(s) & hmask;
-    while (hkey[h] != s) h = (h + 1) & hmask;
-    if (hflag[h]) continue;
-    const int part = slot_part(s, p.G);
-    const bool is_read = (e % WR) >= p.W;
-    const int pos = is_read ? base[part] + cnt_w[part] + atomicAdd(&fill_r[part], 1)
-                            : base[part] + atomicAdd(&fill_w[part], 1);
-    rec[pos] = make_int4(int(s), meta_of(e), __float_as_int(ent_w[e]), 1);
+  // single-use entries: per-warp positions
+  for (int e = e_lo + lane; e < e_hi; e += 32) {
+    const uint8_t key = ent_key[e];
+    if (key == 0xff || key % 3 == 2) continue;
+    const int pos = atomicAdd(&off[warp * NK + key], 1);
+    rec[pos] = make_int4(int(ent_slot[e]), meta_of(e), __float_as_int(ent_w[e]), 1);
   }
+  // multi-use entries: in sorted order, chains
   for (int i = tid; i < n_multi; i += blockDim.x) {
     const int e = mlist[i];
     const uint32_t s = ent_slot[e];
     const int part = slot_part(s, p.G);
-    const int pos = base[part] + cnt_w[part] + cnt_r[part] + (i - mbase[part]);
+    const int pos = kbase[part * 3 + 2] + (i - mbase[part]);
     int len = 0;
     if (i == 0 || ent_slot[mlist[i - 1]] != s) {
       int j = i + 1;
@@ -470,27 +615,33 @@ k_merge_plan(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   // per part g: single writes [3g, 3g+1), single reads [3g+1, 3g+2), multi-use
   // chains [3g+2, 3g+3); entry 3G = end
   int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (3 * p.G + 1);
-  for (int g = tid; g < p.G; g += blockDim.x) {
-    roff[3 * g] = base[g];
-    roff[3 * g + 1] = base[g] + cnt_w[g];
-    roff[3 * g + 2] = base[g] + cnt_w[g] + cnt_r[g];
-  }
-  if (tid == 0) roff[3 * p.G] = base[p.G];
+  for (int kk = tid; kk < NK; kk += blockDim.x) roff[kk] = kbase[kk];
+  if (tid == 0) roff[NK] = misc[1];
   // the recurrence adds every read into o with reductions: start from zero
   float4* o4 = reinterpret_cast<float4*>(io.o + (size_t(bh) * p.T + t0 + s0) * p.dv);
   const int n4 = np * p.dv / 4;
   for (int i = tid; i < n4; i += blockDim.x) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-cudaError_t launch_merge_plan(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
-                              cudaStream_t s) {
-  const size_t smem = merge_smem_bytes(p, p.merge_warps);
-  cudaError_t e = cudaFuncSetAttribute(k_merge_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+cudaError_t launch_merge(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
+                         cudaStream_t s) {
+  const size_t smem = merge_smem_bytes(p, kMergeWarps);
+  cudaError_t e = cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  const int nb = (tlen + p.P - 1) / p.P;
-  dim3 grid(nb, p.BH);
-  k_merge_plan<<<grid, kMergeThreads, smem, s>>>(p, io, t0, tlen, st);
+  dim3 grid((tlen + kMergeSteps - 1) / kMergeSteps, p.BH);
+  k_merge<<<grid, kMergeWarps * 32, smem, s>>>(p, io, t0, tlen, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevStatus* st,
+                        cudaStream_t s) {
+  const size_t smem = plan_smem_bytes(p);
+  cudaError_t e = cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((tlen + p.P - 1) / p.P, p.BH);
+  k_plan<<<grid, kMergeThreads, smem, s>>>(p, io, t0, tlen, st);
   return cudaGetLastError();
 }
 

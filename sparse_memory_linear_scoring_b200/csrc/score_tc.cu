@@ -66,7 +66,7 @@ __host__ __device__ inline TcLayout tc_layout(const Plan& p) {
   L.vals = o; o += uint32_t(p.C) * kTileM * 4;
   L.idx = o; o += uint32_t(p.C) * kTileM * 2;
   o = (o + 15) & ~15u;
-  L.hist = o; o += kBuckets * kTileM * 2;
+  L.hist = o; o += 2 * (kBuckets / 4) * kTileM * 4;
   o = (o + 15) & ~15u;
   L.bars = o; o += 16 * 8;
   L.total = o + 1024;  // slack for 1024-byte alignment of the dynamic base
@@ -195,7 +195,7 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
   unsigned char* sB = smem + L.b;
   float* vals = reinterpret_cast<float*>(smem + L.vals);
   uint16_t* idxs = reinterpret_cast<uint16_t*>(smem + L.idx);
-  uint16_t* hist = reinterpret_cast<uint16_t*>(smem + L.hist);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);  // [2][16][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* full = bars;       // [2] TMA -> MMA
   uint64_t* empty = bars + 2;  // [2] MMA -> TMA
@@ -363,29 +363,55 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       } else {
         // exact top-k of the kept scores, sorted: bucket by value, keep the
         // buckets that hold the k best, sort inside the multi-entry buckets
+        // bucket counts packed 4 per word ([16][128] words, one byte each);
+        // two histograms (even / odd candidates) halve the update chains
+        const float* __restrict__ cv = vals + row;
+        uint32_t* __restrict__ h0 = hist + row;
+        uint32_t* __restrict__ h1 = hist + 16 * kTileM + row;
         float vmin = INFINITY, vmax = -INFINITY;
+#pragma unroll 4
         for (int i = 0; i < cnt; ++i) {
-          const float x = vals[i * kTileM + row];
+          const float x = cv[i * kTileM];
           vmin = fminf(vmin, x);
           vmax = fmaxf(vmax, x);
         }
         const float scale = vmax > vmin ? float(kBuckets) / (vmax - vmin) : 0.f;
-        for (int b = 0; b < kBuckets; ++b) hist[b * kTileM + row] = 0;
-        for (int i = 0; i < cnt; ++i) {
-          const int b = min(kBuckets - 1, int((vals[i * kTileM + row] - vmin) * scale));
-          hist[b * kTileM + row] += 1;
+        auto bucket = [&](float x) { return min(kBuckets - 1, int((x - vmin) * scale)); };
+#pragma unroll
+        for (int w = 0; w < kBuckets / 4; ++w) {
+          h0[w * kTileM] = 0u;
+          h1[w * kTileM] = 0u;
         }
-        int bstar = kBuckets - 1, cum = 0;
-        for (int b = kBuckets - 1; b >= 0; --b) {
-          cum += hist[b * kTileM + row];
-          bstar = b;
-          if (cum >= k) break;
+        int i2 = 0;
+        for (; i2 + 1 < cnt; i2 += 2) {
+          const int b0 = bucket(cv[i2 * kTileM]), b1 = bucket(cv[(i2 + 1) * kTileM]);
+          h0[(b0 >> 2) * kTileM] += 1u << ((b0 & 3) * 8);
+          h1[(b1 >> 2) * kTileM] += 1u << ((b1 & 3) * 8);
         }
+        if (i2 < cnt) {
+          const int b0 = bucket(cv[i2 * kTileM]);
+          h0[(b0 >> 2) * kTileM] += 1u << ((b0 & 3) * 8);
+        }
+        // counts never exceed the capacity (< 256), so bytes add without carry
+        int bstar = 0, cum = 0;
+        for (int w = kBuckets / 4 - 1; w >= 0 && cum < k; --w) {
+          const uint32_t c4 = h0[w * kTileM] + h1[w * kTileM];
+          for (int j = 3; j >= 0; --j) {
+            cum += (c4 >> (8 * j)) & 255u;
+            if (cum >= k) { bstar = 4 * w + j; break; }
+          }
+        }
+        // write offsets (bytes) for buckets >= bstar into h0
         int run = 0;
-        for (int b = kBuckets - 1; b >= bstar; --b) {
-          const int hb = hist[b * kTileM + row];
-          hist[b * kTileM + row] = uint16_t(run);
-          run += hb;
+        for (int w = kBuckets / 4 - 1; w >= (bstar >> 2); --w) {
+          const uint32_t c4 = h0[w * kTileM] + h1[w * kTileM];
+          uint32_t o4 = 0;
+          for (int j = 3; j >= 0; --j) {
+            if (4 * w + j < bstar) continue;
+            o4 |= uint32_t(run) << (8 * j);
+            run += (c4 >> (8 * j)) & 255u;
+          }
+          h0[w * kTileM] = o4;
         }
         const int nout = run;
         const int ocap = out_capacity(L);
@@ -397,28 +423,31 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
         // codebook ring are free: stage the sorted list there, column = row
         uint2* out = reinterpret_cast<uint2*>(smem + L.a);
         for (int i = 0; i < cnt && continue_out; ++i) {
-          const float x = vals[i * kTileM + row];
-          const int b = min(kBuckets - 1, int((x - vmin) * scale));
+          const float x = cv[i * kTileM];
+          const int b = bucket(x);
           if (b >= bstar) {
-            const int pos = hist[b * kTileM + row];
-            hist[b * kTileM + row] = uint16_t(pos + 1);
+            const uint32_t w4 = h0[(b >> 2) * kTileM];
+            const int pos = int((w4 >> ((b & 3) * 8)) & 255u);
+            h0[(b >> 2) * kTileM] = w4 + (1u << ((b & 3) * 8));
             out[pos * kTileM + row] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
           }
         }
         if (continue_out) {
-          int prev = 0;
-          for (int b = kBuckets - 1; b >= bstar; --b) {
-            const int end = hist[b * kTileM + row];
-            for (int i = prev + 1; i < end; ++i) {
-              const uint2 x = out[i * kTileM + row];
+          // the list is sorted across buckets; one insertion pass fixes the
+          // order inside buckets (few moves: only same-bucket entries invert)
+          uint2 last = out[row];
+          for (int i = 1; i < nout; ++i) {
+            const uint2 x = out[i * kTileM + row];
+            if (before(x, last)) {
               int j2 = i - 1;
-              while (j2 >= prev && before(x, out[j2 * kTileM + row])) {
+              while (j2 >= 0 && before(x, out[j2 * kTileM + row])) {
                 out[(j2 + 1) * kTileM + row] = out[j2 * kTileM + row];
                 --j2;
               }
               out[(j2 + 1) * kTileM + row] = x;
+            } else {
+              last = x;
             }
-            prev = end;
           }
           uint4* g = reinterpret_cast<uint4*>(a.surv + hr * C);
           int i = 0;

@@ -6,9 +6,10 @@
 //      candidate lists (tensor cores for bf16 shapes they cover, else CUDA
 //      cores; rows the tensor-core filter could not settle are redone exactly
 //      on CUDA cores);
-//   2. merge_plan: top-W / top-R lists with softmax weights, grouped into the
-//      recurrence's per-part plan (or written out as lists for sdm_select);
-//   3. recur: the gated delta writes and the reads, in time order.
+//   2. merge: top-W / top-R lists with softmax weights (into the workspace, or
+//      the caller's lists for sdm_select);
+//   3. plan: the lists grouped into the recurrence's per-part records;
+//   4. recur: the gated delta writes and the reads, in time order.
 #include <limits.h>
 #include <stdint.h>
 #include <string.h>
@@ -19,6 +20,7 @@ namespace sdm {
 
 size_t score_simt_smem(const Plan& p);
 size_t merge_smem_bytes(const Plan& p, int warps);
+size_t plan_smem_bytes(const Plan& p);
 size_t recur_smem_bytes(const Plan& p);
 size_t score_tc_smem(const Plan& p);
 int score_tc_capacity(const sdm_dims* d);
@@ -87,7 +89,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
   p->G = G;
   // time chunk: bounded workspace
   const size_t per_step = size_t(p->BH) * (4 * 4 + size_t(4) * p->C * 8 + 4 * 4 +
-                                           size_t(p->W + p->R) * 16) +
+                                           size_t(p->W + p->R) * (16 + 8)) +
                           (size_t(p->BH) * (3 * p->G + 1) * 4 + size_t(P) - 1) / size_t(P);
   const long long Tround = ((long long)(p->T > 0 ? p->T : 1) + P - 1) / P * P;
   long long Tc = (long long)(kChunkBudget / per_step) / P * P;
@@ -96,13 +98,12 @@ int make_plan(const sdm_dims* d, Plan* p) {
   p->Tc = int(Tc);
   p->nchunks = p->T == 0 ? 0 : int((p->T + Tc - 1) / Tc);
   p->nblk = int((Tc + P - 1) / P);
-  int mw = kMergeThreads / 32;
-  while (mw > 1 && merge_smem_bytes(*p, mw) > kMaxSmem) mw >>= 1;
-  p->merge_warps = mw;
-  p->merge_smem = merge_smem_bytes(*p, mw);
+  p->merge_smem = merge_smem_bytes(*p, kMergeWarps);
+  p->plan_smem = plan_smem_bytes(*p);
   p->recur_smem = recur_smem_bytes(*p);
   p->score_smem = p->tc ? score_tc_smem(*p) : score_simt_smem(*p);
-  if (p->merge_smem > kMaxSmem || p->recur_smem > kMaxSmem || p->score_smem > kMaxSmem)
+  if (p->merge_smem > kMaxSmem || p->plan_smem > kMaxSmem || p->recur_smem > kMaxSmem ||
+      p->score_smem > kMaxSmem)
     return SDM_ERR_UNSUPPORTED;
   const size_t nhr = size_t(p->BH) * p->Tc * 4;
   size_t o = 0;
@@ -110,6 +111,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
   p->off_cnt = o; o = align256(o + nhr * 4);
   p->off_surv = o; o = align256(o + nhr * p->C * 8);
   p->off_redo = o; o = align256(o + nhr * 4);
+  p->off_lists = o; o = align256(o + size_t(p->BH) * p->Tc * (p->W + p->R) * 8);
   p->off_rec = o; o = align256(o + size_t(p->BH) * p->nblk * p->E * 16);
   p->off_roff = o; o = align256(o + size_t(p->BH) * p->nblk * (3 * p->G + 1) * 4);
   p->total = o;
@@ -142,6 +144,7 @@ struct Carve {
   int* cnt;
   uint2* surv;
   int* redo;
+  int32_t* iw; float* ww; int32_t* ir; float* wr;  // this chunk's lists
   int4* rec;
   int* roff;
 };
@@ -153,6 +156,14 @@ static Carve carve(const Plan& p, void* ws) {
   c.cnt = reinterpret_cast<int*>(b + p.off_cnt);
   c.surv = reinterpret_cast<uint2*>(b + p.off_surv);
   c.redo = reinterpret_cast<int*>(b + p.off_redo);
+  {
+    const size_t rows = size_t(p.BH) * p.Tc;
+    char* l = b + p.off_lists;
+    c.iw = reinterpret_cast<int32_t*>(l);
+    c.ww = reinterpret_cast<float*>(l + rows * p.W * 4);
+    c.ir = reinterpret_cast<int32_t*>(l + rows * p.W * 8);
+    c.wr = reinterpret_cast<float*>(l + rows * p.W * 8 + rows * p.R * 4);
+  }
   c.rec = reinterpret_cast<int4*>(b + p.off_rec);
   c.roff = reinterpret_cast<int*>(b + p.off_roff);
   return c;
@@ -215,21 +226,31 @@ static int forward_impl(const void* q, const void* k, const void* v, const float
     return cudaEventRecord(static_cast<cudaEvent_t>(events[j]), s) == cudaSuccess;
   };
   if (launch_init(p, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
-  MergeIO io;
-  memset(&io, 0, sizeof(io));
-  io.mode = 0;
-  io.surv_cnt = c.cnt;
-  io.surv = c.surv;
-  io.rec = c.rec;
-  io.roff = c.roff;
-  io.o = o_out;
+  MergeIO mio;
+  memset(&mio, 0, sizeof(mio));
+  mio.surv_cnt = c.cnt;
+  mio.surv = c.surv;
+  mio.out_iw = c.iw; mio.out_ww = c.ww; mio.out_ir = c.ir; mio.out_wr = c.wr;
+  mio.list_T = p.Tc;
+  mio.list_t0 = 0;
+  mio.sorted = 0;
+  PlanIO pio;
+  memset(&pio, 0, sizeof(pio));
+  pio.iw = c.iw; pio.ww = c.ww; pio.ir = c.ir; pio.wr = c.wr;
+  pio.list_T = p.Tc;
+  pio.list_t0 = 0;
+  pio.validate = 0;
+  pio.rec = c.rec;
+  pio.roff = c.roff;
+  pio.o = o_out;
   for (int ch = 0; ch < p.nchunks; ++ch) {
     const int t0 = ch * p.Tc;
     const int tlen = (p.T - t0 < p.Tc) ? p.T - t0 : p.Tc;
     if (!mark(4 * ch)) return SDM_ERR_CUDA;
     if (score_chunk(p, c, q, k, C1, C2, t0, tlen, s) != cudaSuccess) return SDM_ERR_CUDA;
     if (!mark(4 * ch + 1)) return SDM_ERR_CUDA;
-    if (launch_merge_plan(p, io, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
+    if (launch_merge(p, mio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
+    if (launch_plan(p, pio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
     if (!mark(4 * ch + 2)) return SDM_ERR_CUDA;
     if (launch_recur(p, v, alpha, beta, M_inout, o_out, c.rec, c.roff, t0, tlen, c.st, s) !=
         cudaSuccess)
@@ -260,7 +281,7 @@ extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
   Plan p;
   const int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
-  const int64_t per_chunk = (p.tc ? 3 : 1) + 2;
+  const int64_t per_chunk = (p.tc ? 3 : 1) + 3;
   const int64_t vals[7] = {p.tc, p.C, p.P, p.G, p.Tc, p.nchunks, 1 + per_chunk * p.nchunks};
   for (int i = 0; i < n && i < 7; ++i) out[i] = vals[i];
   return SDM_OK;
@@ -279,17 +300,19 @@ extern "C" int sdm_select(const void* q, const void* k, const void* C1, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Carve c = carve(p, workspace);
   if (launch_init(p, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
-  MergeIO io;
-  memset(&io, 0, sizeof(io));
-  io.mode = 1;
-  io.surv_cnt = c.cnt;
-  io.surv = c.surv;
-  io.out_iw = idx_w; io.out_ww = w_w; io.out_ir = idx_r; io.out_wr = w_r;
+  MergeIO mio;
+  memset(&mio, 0, sizeof(mio));
+  mio.surv_cnt = c.cnt;
+  mio.surv = c.surv;
+  mio.out_iw = idx_w; mio.out_ww = w_w; mio.out_ir = idx_r; mio.out_wr = w_r;
+  mio.list_T = p.T;
+  mio.sorted = 1;
   for (int ch = 0; ch < p.nchunks; ++ch) {
     const int t0 = ch * p.Tc;
     const int tlen = (p.T - t0 < p.Tc) ? p.T - t0 : p.Tc;
+    mio.list_t0 = t0;
     if (score_chunk(p, c, q, k, C1, C2, t0, tlen, s) != cudaSuccess) return SDM_ERR_CUDA;
-    if (launch_merge_plan(p, io, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
+    if (launch_merge(p, mio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
   }
   return SDM_OK;
 }
@@ -308,17 +331,19 @@ extern "C" int sdm_recur(const void* v, const float* alpha, const float* beta,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Carve c = carve(p, workspace);
   if (launch_init(p, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
-  MergeIO io;
-  memset(&io, 0, sizeof(io));
-  io.mode = 2;
-  io.in_iw = idx_w; io.in_ww = w_w; io.in_ir = idx_r; io.in_wr = w_r;
-  io.rec = c.rec;
-  io.roff = c.roff;
-  io.o = o_out;
+  PlanIO pio;
+  memset(&pio, 0, sizeof(pio));
+  pio.iw = idx_w; pio.ww = w_w; pio.ir = idx_r; pio.wr = w_r;
+  pio.list_T = p.T;
+  pio.validate = 1;
+  pio.rec = c.rec;
+  pio.roff = c.roff;
+  pio.o = o_out;
   for (int ch = 0; ch < p.nchunks; ++ch) {
     const int t0 = ch * p.Tc;
     const int tlen = (p.T - t0 < p.Tc) ? p.T - t0 : p.Tc;
-    if (launch_merge_plan(p, io, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
+    pio.list_t0 = t0;
+    if (launch_plan(p, pio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
     if (launch_recur(p, v, alpha, beta, M_inout, o_out, c.rec, c.roff, t0, tlen, c.st, s) !=
         cudaSuccess)
       return SDM_ERR_CUDA;

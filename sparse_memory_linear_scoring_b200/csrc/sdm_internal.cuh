@@ -31,7 +31,9 @@ constexpr int kTargetCtas = SDM_TARGET_CTAS;  // recurrence CTAs aimed for (2 x 
 constexpr int kMaxParts = 64;           // slot parts per head in the recurrence
 constexpr int kMaxBlockEntries = 8192;  // list entries per (head, block) in a plan
 constexpr size_t kChunkBudget = size_t(1) << 30;  // workspace bytes per time chunk
-constexpr int kMergeThreads = 512;
+constexpr int kMergeThreads = 512;     // plan kernel
+constexpr int kMergeWarps = 8;          // merge kernel: warps per CTA
+constexpr int kMergeSteps = 16;         // merge kernel: steps per CTA
 constexpr int kRecurThreads = SDM_RECUR_THREADS;
 constexpr int kRecurUnroll = SDM_RECUR_UNROLL;
 
@@ -49,10 +51,9 @@ struct Plan {
   int E;       // list entries per plan block = P * (W + R)
   int G;       // slot parts per head
   int ncW, nfW, ncR, nfR;  // staircase / frontier sizes of the merge
-  int merge_warps;         // warps doing merges inside a merge_plan CTA
-  size_t merge_smem, recur_smem, score_smem;
+  size_t merge_smem, plan_smem, recur_smem, score_smem;
   // workspace byte offsets
-  size_t off_status, off_cnt, off_surv, off_redo, off_rec, off_roff, total;
+  size_t off_status, off_cnt, off_surv, off_redo, off_lists, off_rec, off_roff, total;
 };
 
 // Workspace status words.
@@ -139,19 +140,28 @@ cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const v
                             int* redo_rows, DevStatus* st, cudaStream_t s);
 bool score_tc_supported(const sdm_dims* d);
 
+// Lists of (slot, weight) pairs: iw/ww [rows][W], ir/wr [rows][R]; a step's
+// row is bh * list_T + list_t0 + (step within the chunk).
 struct MergeIO {
-  // mode 0: survivors -> plan;  1: survivors -> lists;  2: lists -> plan
-  int mode;
   const int* surv_cnt;
   const uint2* surv;
-  const int32_t* in_iw; const float* in_ww; const int32_t* in_ir; const float* in_wr;
   int32_t* out_iw; float* out_ww; int32_t* out_ir; float* out_wr;
+  int list_T, list_t0;
+  int sorted;  // write each list in rank order
+};
+cudaError_t launch_merge(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
+                         cudaStream_t s);
+
+struct PlanIO {
+  const int32_t* iw; const float* ww; const int32_t* ir; const float* wr;
+  int list_T, list_t0;
+  int validate;  // flag out-of-range slots (caller lists)
   int4* rec;
   int* roff;
   float* o;
 };
-cudaError_t launch_merge_plan(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
-                              cudaStream_t s);
+cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevStatus* st,
+                        cudaStream_t s);
 
 cudaError_t launch_recur(const Plan& p, const void* v, const float* alpha, const float* beta,
                          float* M, float* o, const int4* rec, const int* roff, int t0, int tlen,

@@ -133,6 +133,22 @@ def test_tensor_core_scoring_shapes(shape):
     _check_forward(cfg, inp, ref)
 
 
+@pytest.mark.parametrize("base", [
+    config(1).with_(B=1, H=2, T=200, n_sub=256, k=32, W=64, R=64, m0_sd=0.5),
+    config(0).with_(B=1, H=2, T=150, m0_sd=0.5),
+], ids=["bf16-tensor-core", "fp32"])
+def test_duplicate_codebook_rows(base):
+    """Duplicated codebook rows make exact score ties at every rank: the lower
+    index must win in each half and among slots, on the GPU as in the oracle."""
+    inp = gen_inputs(base)
+    for name in ("C1", "C2"):
+        c = inp[name].clone()
+        c[:, 1::2] = c[:, 0::2]
+        inp[name] = c
+    ref = oracle_full(inp, base, lists=True)
+    _check_forward(base, inp, ref)
+
+
 def test_fp32_wide_rows():
     cfg = config(0).with_(B=2, H=3, T=200, d_v=128, d_qk=24, n_sub=16, k=6, W=20, R=12,
                           m0_sd=1.0)
