@@ -538,9 +538,24 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
     tot[kk] = t;
   }
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0, macc = 0;
-    for (int kk = 0; kk < NK; ++kk) {
+  if (warp == 0) {
+    // exclusive scans over the keys (and over the parts' multi counts), one warp
+    const int per = (NK + 31) / 32;
+    const int k0 = lane * per, k1 = min(NK, k0 + per);
+    int sa = 0, sm = 0;
+    for (int kk = k0; kk < k1; ++kk) {
+      sa += tot[kk];
+      if (kk % 3 == 2) sm += tot[kk];
+    }
+    int ia = sa, im = sm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, ia, o);
+      const int ym = __shfl_up_sync(0xffffffffu, im, o);
+      if (lane >= o) { ia += ya; im += ym; }
+    }
+    int acc = ia - sa, macc = im - sm;
+    for (int kk = k0; kk < k1; ++kk) {
       kbase[kk] = acc;
       acc += tot[kk];
       if (kk % 3 == 2) {
@@ -548,7 +563,7 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
         macc += tot[kk];
       }
     }
-    misc[1] = acc;
+    if (lane == 31) misc[1] = ia;
   }
   __syncthreads();
   for (int kk = tid; kk < NK; kk += blockDim.x) {
@@ -569,7 +584,24 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
       const uint32_t s = ent_slot[e];
       return (uint64_t(slot_part(s, p.G)) << 46) | (uint64_t(s) << 14) | uint64_t(e);
     };
-    for (int size = 2; size <= S; size <<= 1) {
+    if (S <= 512) {
+      // few multi-use entries (the usual case): one warp sorts them
+      if (warp == 0) {
+        for (int size = 2; size <= S; size <<= 1) {
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = lane; i < (S >> 1); i += 32) {
+              const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
+              const int hi = lo + stride;
+              const uint16_t x = mlist[lo], y = mlist[hi];
+              const uint64_t kx = mkey(x), ky = mkey(y);
+              const bool asc = (lo & size) == 0;
+              if (asc ? (kx > ky) : (kx < ky)) { mlist[lo] = y; mlist[hi] = x; }
+            }
+            __syncwarp();
+          }
+        }
+      }
+    } else for (int size = 2; size <= S; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
         for (int i = tid; i < (S >> 1); i += blockDim.x) {
           const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));

@@ -186,9 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
            const __grid_constant__ CUtensorMap mc1, const __grid_constant__ CUtensorMap mc2,
            TcArgs a) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the swizzled tiles, by offset arithmetic on the
+  // shared array itself so that every access stays a shared-memory access
+  unsigned char* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
   const Plan& p = a.p;
   const TcLayout L = tc_layout(p);
   unsigned char* sA = smem + L.a;
@@ -433,30 +434,23 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
           }
         }
         if (continue_out) {
-          // the list is sorted across buckets; one insertion pass fixes the
-          // order inside buckets (few moves: only same-bucket entries invert)
-          uint2 last = out[row];
-          for (int i = 1; i < nout; ++i) {
+          // The staged list is ordered by bucket; an entry's final rank is its
+          // bucket's start plus the entries of its own bucket that precede it.
+          // Entries ranked below k go straight to their slot in the output.
+          uint2* g = a.surv + hr * C;
+          for (int i = 0; i < nout; ++i) {
             const uint2 x = out[i * kTileM + row];
-            if (before(x, last)) {
-              int j2 = i - 1;
-              while (j2 >= 0 && before(x, out[j2 * kTileM + row])) {
-                out[(j2 + 1) * kTileM + row] = out[j2 * kTileM + row];
-                --j2;
-              }
-              out[(j2 + 1) * kTileM + row] = x;
-            } else {
-              last = x;
-            }
+            const int b = bucket(__uint_as_float(x.x));
+            const int end = int((h0[(b >> 2) * kTileM] >> ((b & 3) * 8)) & 255u);
+            const int bn = b + 1;
+            const int start = bn >= kBuckets
+                                  ? 0
+                                  : int((h0[(bn >> 2) * kTileM] >> ((bn & 3) * 8)) & 255u);
+            int rank = start;
+            for (int j = start; j < end; ++j) rank += before(out[j * kTileM + row], x) ? 1 : 0;
+            if (rank < k) g[rank] = x;
           }
-          uint4* g = reinterpret_cast<uint4*>(a.surv + hr * C);
-          int i = 0;
-          for (; i + 1 < nout; i += 2) {
-            const uint2 x0 = out[i * kTileM + row], x1 = out[(i + 1) * kTileM + row];
-            g[i >> 1] = make_uint4(x0.x, x0.y, x1.x, x1.y);
-          }
-          if (i < nout) a.surv[hr * C + i] = out[i * kTileM + row];
-          a.cnt[hr] = nout;
+          a.cnt[hr] = k;
         }
       }
     }
