@@ -162,9 +162,12 @@ def run_sdm(args, cfg, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    from sparse_memory_linear_scoring_b200.parallel import max_over_ranks, shard_batch
     dims = sdm.make_dims(**cfg.dims())
     plan = sdm.query_plan(dims)
-    inp = gen_inputs(cfg, b0=rank * cfg.B)
+    # weak scaling: rank r owns batch rows [r*B, (r+1)*B) of a world*B batch
+    b0, _ = shard_batch(cfg.B * world, world, rank)
+    inp = gen_inputs(cfg, b0=b0)
     dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
     d = {n: inp[n].to(dev, dt).contiguous() for n in ("q", "k", "v", "C1", "C2")}
     for n in ("alpha", "beta"):
@@ -222,12 +225,8 @@ def run_sdm(args, cfg, rank, world, local_rank):
     st, info = sdm.device_status()
     if st != 0:
         raise RuntimeError("device status %d (info %d) after timing" % (st, info))
-    t_max = total
-    if world > 1:
-        tt = torch.tensor([total] + phase, dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt[0])
-        phase = [float(x) for x in tt[1:]]
+    t_max = max_over_ranks(total, dev)
+    phase = [max_over_ranks(x, dev) for x in phase]
 
     # ---- end to end through the public API: pinned host inputs -> device ->
     # forward -> o back to pinned host memory, every step
@@ -264,10 +263,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
             s1.record()
             s1.synchronize()
             et += s0.elapsed_time(s1)
-        if world > 1:
-            tt = torch.tensor([et], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            et = float(tt[0])
+        et = max_over_ranks(et, dev)
         e2e = {"value": world * cfg.BH * cfg.T * args.steps / (et / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
