@@ -12,7 +12,9 @@
 //   warp 1      allocates 512 TMEM columns; one lane issues
 //               tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32, M=128, N=256,
 //               K=16 steps) into two 256-column TMEM buffers;
-//   warps 2..5  epilogue, one thread per token row (TMEM lane): tcgen05.ld the
+//   warps 2..17 epilogue, kQ = 4 threads per token row (the kQ warps whose
+//               warp index is equal mod 4 share one 32-lane TMEM quarter; each
+//               takes a quarter of every 256-column tile): tcgen05.ld the
 //               row's scores, keep those above a threshold tau taken from the
 //               row's own score mean and deviation (first 512 columns), then
 //               select the exact top-k of the kept scores and write them sorted
@@ -36,7 +38,9 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
 constexpr int kKAtom = 64;           // bf16 elements per 128-byte swizzle row
-constexpr int kThreads = 192;
+constexpr int kQ = 4;                // epilogue threads per token row
+constexpr int kEpiThreads = kQ * kTileM;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kBuckets = 64;         // final-selection buckets per row
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 constexpr uint32_t kATileBytes = kTileM * 128;   // one 64-column chunk of the token tile
@@ -53,7 +57,7 @@ struct TcArgs {
 };
 
 struct TcLayout {
-  uint32_t a, b, vals, idx, hist, bars, total;
+  uint32_t a, b, vals, idx, hist, rows, bars, total;
   int nkc;
 };
 
@@ -66,9 +70,10 @@ __host__ __device__ inline TcLayout tc_layout(const Plan& p) {
   L.vals = o; o += uint32_t(p.C) * kTileM * 4;
   L.idx = o; o += uint32_t(p.C) * kTileM * 2;
   o = (o + 15) & ~15u;
-  L.hist = o; o += 2 * (kBuckets / 4) * kTileM * 4;
+  L.hist = o; o += (kBuckets / 4) * kTileM * 4;
+  L.rows = o; o += (2 + 4 * kQ) * kTileM * 4;  // per-row count, nout, partial stats
   o = (o + 15) & ~15u;
-  L.bars = o; o += 16 * 8;
+  L.bars = o; o += 16 * 8;  // mbarriers, TMEM address, abort flags
   L.total = o + 1024;  // slack for 1024-byte alignment of the dynamic base
   return L;
 }
@@ -176,6 +181,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// named barrier of the epilogue warps
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
 // (score desc, row asc) order on the output pairs
 __device__ __forceinline__ bool before(uint2 a, uint2 b) {
   const float va = __uint_as_float(a.x), vb = __uint_as_float(b.x);
@@ -196,7 +206,7 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
   unsigned char* sB = smem + L.b;
   float* vals = reinterpret_cast<float*>(smem + L.vals);
   uint16_t* idxs = reinterpret_cast<uint16_t*>(smem + L.idx);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);  // [2][16][128]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);  // [16][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* full = bars;       // [2] TMA -> MMA
   uint64_t* empty = bars + 2;  // [2] MMA -> TMA
@@ -218,11 +228,12 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4 * 32);
+      mbar_init(&tempty[i], kEpiThreads);
     }
     mbar_init(a_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
+    *reinterpret_cast<volatile int*>(bars + 12) = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -297,24 +308,37 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       }
     }
   } else {
-    // ---------------- epilogue: thread = token row = TMEM lane
+    // ---------------- epilogue: kQ threads per token row (= TMEM lane)
     const int q4 = warp & 3;
+    const int sub = (warp - 2) >> 2;  // which kCols-column slice of every tile
     const int row = q4 * 32 + lane;
     const int tl = tile * kTileM + row;
     const bool valid = tl < a.tlen;
     const uint32_t tbase = tmem + (uint32_t(q4 * 32) << 16);
     const int C = p.C;
+    constexpr int kCols = kTileN / kQ;
+    int* rcnt = reinterpret_cast<int*>(smem + L.rows);      // [128] kept count
+    int* rsel = rcnt + kTileM;                              // [128] nout | bstar << 16
+    float* rst = reinterpret_cast<float*>(rsel + kTileM);   // [4][kQ][128] sum, sq, min, max
+    uint32_t* h = hist + row;                               // [16][128] packed byte counts
+    volatile int* epi_abort = reinterpret_cast<volatile int*>(bars + 12);
     float v[32];
-    bool ok = true;
+    if (sub == 0) {
+      rcnt[row] = 0;
+#pragma unroll
+      for (int w = 0; w < kBuckets / 4; ++w) h[w * kTileM] = 0u;
+    }
     // statistics of the first (up to) two tiles
     const int nstat = ntiles < 2 ? ntiles : 2;
     float sum = 0.f, sq = 0.f;
+    bool ok = true;
     for (int j = 0; j < nstat && ok; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&tfull[j], 0, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      for (int c = 0; c < kTileN / 32; ++c) {
-        tmem_ld32(tbase + uint32_t(j * kTileN + c * 32), v);
+#pragma unroll 1
+      for (int c = 0; c < kCols / 32; ++c) {
+        tmem_ld32(tbase + uint32_t(j * kTileN + sub * kCols + c * 32), v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           sum += v[i];
@@ -322,14 +346,29 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
         }
       }
     }
-    const float m = float(nstat * kTileN);
-    const float mu = sum / m;
-    const float var = fmaxf(sq / m - mu * mu, 0.f);
-    const float sd = sqrtf(var);
+    if (!ok) *epi_abort = 1;
+    rst[(0 * kQ + sub) * kTileM + row] = sum;
+    rst[(1 * kQ + sub) * kTileM + row] = sq;
+    epi_sync();
+    ok = !*epi_abort;
     const bool keep_all = !(a.z > -1e30f);
-    const float tau = keep_all ? -INFINITY : mu + a.z * sd;
-    bool redo = !keep_all && !(sd > 0.f);
-    int cnt = 0;
+    float tau = -INFINITY;
+    bool redo = false;
+    {
+      float S = 0.f, S2 = 0.f;
+#pragma unroll
+      for (int j = 0; j < kQ; ++j) {
+        S += rst[(0 * kQ + j) * kTileM + row];
+        S2 += rst[(1 * kQ + j) * kTileM + row];
+      }
+      const float m = float(nstat * kTileN);
+      const float mu = S / m;
+      const float sd = sqrtf(fmaxf(S2 / m - mu * mu, 0.f));
+      if (!keep_all) tau = mu + a.z * sd;
+      redo = !keep_all && !(sd > 0.f);
+    }
+    // filter: append the kept scores of this thread's columns to the row's list
+    float kmin = INFINITY, kmax = -INFINITY;
     for (int j = 0; j < ntiles && ok; ++j) {
       const int s = j & 1;
       if (j >= 2) {
@@ -337,122 +376,122 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
         if (!ok) break;
         tc_fence_after();
       }
-      for (int c = 0; c < kTileN / 32; ++c) {
-        tmem_ld32(tbase + uint32_t(s * kTileN + c * 32), v);
-        const int col0 = j * kTileN + c * 32;
+#pragma unroll 1
+      for (int c = 0; c < kCols / 32; ++c) {
+        tmem_ld32(tbase + uint32_t(s * kTileN + sub * kCols + c * 32), v);
+        const int col0 = j * kTileN + sub * kCols + c * 32;
+        uint32_t mask = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool keep = v[i] >= tau;
-          if (keep && cnt < C) {
-            vals[cnt * kTileM + row] = v[i];
-            idxs[cnt * kTileM + row] = uint16_t(col0 + i);
+        for (int i = 0; i < 32; ++i) mask |= (v[i] >= tau ? 1u : 0u) << i;
+        if (mask) {
+          int pos = atomicAdd(&rcnt[row], __popc(mask));
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if ((mask >> i) & 1u) {
+              if (pos < C) {
+                vals[pos * kTileM + row] = v[i];
+                idxs[pos * kTileM + row] = uint16_t(col0 + i);
+              }
+              kmin = fminf(kmin, v[i]);
+              kmax = fmaxf(kmax, v[i]);
+              ++pos;
+            }
           }
-          cnt += keep ? 1 : 0;
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[s]);
     }
-    if (!ok) {
-      if (lane == 0) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
-    } else if (valid) {
-      const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
-      const int k = p.k;
-      bool continue_out = true;
-      if (redo || cnt < k || cnt > C) {
-        a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
-      } else {
-        // exact top-k of the kept scores, sorted: bucket by value, keep the
-        // buckets that hold the k best, sort inside the multi-entry buckets
-        // bucket counts packed 4 per word ([16][128] words, one byte each);
-        // two histograms (even / odd candidates) halve the update chains
-        const float* __restrict__ cv = vals + row;
-        uint32_t* __restrict__ h0 = hist + row;
-        uint32_t* __restrict__ h1 = hist + 16 * kTileM + row;
-        float vmin = INFINITY, vmax = -INFINITY;
-#pragma unroll 4
-        for (int i = 0; i < cnt; ++i) {
-          const float x = cv[i * kTileM];
-          vmin = fminf(vmin, x);
-          vmax = fmaxf(vmax, x);
-        }
-        const float scale = vmax > vmin ? float(kBuckets) / (vmax - vmin) : 0.f;
-        auto bucket = [&](float x) { return min(kBuckets - 1, int((x - vmin) * scale)); };
+    if (!ok) *epi_abort = 1;
+    rst[(2 * kQ + sub) * kTileM + row] = kmin;
+    rst[(3 * kQ + sub) * kTileM + row] = kmax;
+    epi_sync();
+    ok = !*epi_abort;
+    if (!ok && threadIdx.x == 64) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
+    // exact top-k of the kept scores, sorted: bucket by value, keep the buckets
+    // that hold the k best, rank the entries inside each bucket
+    const int cnt = rcnt[row];
+    const int k = p.k;
+    const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
+    bool go = ok && valid && !redo && cnt >= k && cnt <= C;
+    if (ok && valid && !go && sub == 0) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+    float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kBuckets / 4; ++w) {
-          h0[w * kTileM] = 0u;
-          h1[w * kTileM] = 0u;
-        }
-        int i2 = 0;
-        for (; i2 + 1 < cnt; i2 += 2) {
-          const int b0 = bucket(cv[i2 * kTileM]), b1 = bucket(cv[(i2 + 1) * kTileM]);
-          h0[(b0 >> 2) * kTileM] += 1u << ((b0 & 3) * 8);
-          h1[(b1 >> 2) * kTileM] += 1u << ((b1 & 3) * 8);
-        }
-        if (i2 < cnt) {
-          const int b0 = bucket(cv[i2 * kTileM]);
-          h0[(b0 >> 2) * kTileM] += 1u << ((b0 & 3) * 8);
-        }
-        // counts never exceed the capacity (< 256), so bytes add without carry
-        int bstar = 0, cum = 0;
-        for (int w = kBuckets / 4 - 1; w >= 0 && cum < k; --w) {
-          const uint32_t c4 = h0[w * kTileM] + h1[w * kTileM];
-          for (int j = 3; j >= 0; --j) {
-            cum += (c4 >> (8 * j)) & 255u;
-            if (cum >= k) { bstar = 4 * w + j; break; }
-          }
-        }
-        // write offsets (bytes) for buckets >= bstar into h0
-        int run = 0;
-        for (int w = kBuckets / 4 - 1; w >= (bstar >> 2); --w) {
-          const uint32_t c4 = h0[w * kTileM] + h1[w * kTileM];
-          uint32_t o4 = 0;
-          for (int j = 3; j >= 0; --j) {
-            if (4 * w + j < bstar) continue;
-            o4 |= uint32_t(run) << (8 * j);
-            run += (c4 >> (8 * j)) & 255u;
-          }
-          h0[w * kTileM] = o4;
-        }
-        const int nout = run;
-        const int ocap = out_capacity(L);
-        if (nout > ocap) {
-          a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
-          continue_out = false;
-        }
-        // every MMA has completed (the last tfull wait), so the token tile and
-        // codebook ring are free: stage the sorted list there, column = row
-        uint2* out = reinterpret_cast<uint2*>(smem + L.a);
-        for (int i = 0; i < cnt && continue_out; ++i) {
-          const float x = cv[i * kTileM];
-          const int b = bucket(x);
-          if (b >= bstar) {
-            const uint32_t w4 = h0[(b >> 2) * kTileM];
-            const int pos = int((w4 >> ((b & 3) * 8)) & 255u);
-            h0[(b >> 2) * kTileM] = w4 + (1u << ((b & 3) * 8));
-            out[pos * kTileM + row] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
-          }
-        }
-        if (continue_out) {
-          // The staged list is ordered by bucket; an entry's final rank is its
-          // bucket's start plus the entries of its own bucket that precede it.
-          // Entries ranked below k go straight to their slot in the output.
-          uint2* g = a.surv + hr * C;
-          for (int i = 0; i < nout; ++i) {
-            const uint2 x = out[i * kTileM + row];
-            const int b = bucket(__uint_as_float(x.x));
-            const int end = int((h0[(b >> 2) * kTileM] >> ((b & 3) * 8)) & 255u);
-            const int bn = b + 1;
-            const int start = bn >= kBuckets
-                                  ? 0
-                                  : int((h0[(bn >> 2) * kTileM] >> ((bn & 3) * 8)) & 255u);
-            int rank = start;
-            for (int j = start; j < end; ++j) rank += before(out[j * kTileM + row], x) ? 1 : 0;
-            if (rank < k) g[rank] = x;
-          }
-          a.cnt[hr] = k;
+    for (int j = 0; j < kQ; ++j) {
+      vmin = fminf(vmin, rst[(2 * kQ + j) * kTileM + row]);
+      vmax = fmaxf(vmax, rst[(3 * kQ + j) * kTileM + row]);
+    }
+    const float scale = vmax > vmin ? float(kBuckets) / (vmax - vmin) : 0.f;
+    auto bucket = [&](float x) { return min(kBuckets - 1, int((x - vmin) * scale)); };
+    const float* __restrict__ cv = vals + row;
+    if (go) {
+      for (int i = sub; i < cnt; i += kQ) {
+        const int b = bucket(cv[i * kTileM]);
+        atomicAdd(&h[(b >> 2) * kTileM], 1u << ((b & 3) * 8));
+      }
+    }
+    epi_sync();
+    if (go && sub == 0) {
+      // counts never exceed the capacity (< 256), so bytes add without carry
+      int bstar = 0, cum = 0;
+      for (int w = kBuckets / 4 - 1; w >= 0 && cum < k; --w) {
+        const uint32_t c4 = h[w * kTileM];
+        for (int j = 3; j >= 0; --j) {
+          cum += (c4 >> (8 * j)) & 255u;
+          if (cum >= k) { bstar = 4 * w + j; break; }
         }
       }
+      // start offsets (descending bucket order) of the buckets >= bstar
+      int run = 0;
+      for (int w = kBuckets / 4 - 1; w >= (bstar >> 2); --w) {
+        const uint32_t c4 = h[w * kTileM];
+        uint32_t o4 = 0;
+        for (int j = 3; j >= 0; --j) {
+          if (4 * w + j < bstar) continue;
+          o4 |= uint32_t(run) << (8 * j);
+          run += (c4 >> (8 * j)) & 255u;
+        }
+        h[w * kTileM] = o4;
+      }
+      rsel[row] = run | (bstar << 16);
+      if (run > out_capacity(L)) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+    }
+    epi_sync();
+    const int nout = go ? (rsel[row] & 0xffff) : 0;
+    const int bstar = go ? (rsel[row] >> 16) : 0;
+    go = go && nout <= out_capacity(L);
+    // every MMA has completed (each thread waited for the last tile), so the
+    // token tile and codebook ring are free: stage the bucketed list there
+    uint2* out = reinterpret_cast<uint2*>(smem + L.a);
+    if (go) {
+      for (int i = sub; i < cnt; i += kQ) {
+        const float x = cv[i * kTileM];
+        const int b = bucket(x);
+        if (b >= bstar) {
+          const uint32_t old = atomicAdd(&h[(b >> 2) * kTileM], 1u << ((b & 3) * 8));
+          const int pos = int((old >> ((b & 3) * 8)) & 255u);
+          out[pos * kTileM + row] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
+        }
+      }
+    }
+    epi_sync();
+    if (go) {
+      // h now holds each bucket's end; its start is the end of the bucket above.
+      // An entry's final rank is its bucket's start plus the entries of its own
+      // bucket that precede it; entries ranked below k go straight to the output.
+      uint2* g = a.surv + hr * C;
+      for (int i = sub; i < nout; i += kQ) {
+        const uint2 x = out[i * kTileM + row];
+        const int b = bucket(__uint_as_float(x.x));
+        const int end = int((h[(b >> 2) * kTileM] >> ((b & 3) * 8)) & 255u);
+        const int bn = b + 1;
+        const int start =
+            bn >= kBuckets ? 0 : int((h[(bn >> 2) * kTileM] >> ((bn & 3) * 8)) & 255u);
+        int rank = start;
+        for (int j = start; j < end; ++j) rank += before(out[j * kTileM + row], x) ? 1 : 0;
+        if (rank < k) g[rank] = x;
+      }
+      if (sub == 0) a.cnt[hr] = k;
     }
   }
   tc_fence_before();
@@ -522,7 +561,8 @@ bool score_tc_supported(const sdm_dims* d) {
   tmp.dh = dh;
   tmp.C = score_tc_capacity(d);
   const TcLayout L = tc_layout(tmp);
-  return L.total <= 227 * 1024 && out_capacity(L) >= d->k + 16;
+  // per-row bucket counts and offsets are packed bytes: the capacity stays below 256
+  return tmp.C <= 255 && L.total <= 227 * 1024 && out_capacity(L) >= d->k + 16;
 }
 
 cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const void* C1,
