@@ -176,7 +176,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
     del inp
     o = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    nph = 4 * plan["chunks"]
+    nph = 5 * plan["chunks"]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(nph)]
     for e in ev:          # torch creates the CUDA event on its first record
         e.record()
@@ -205,7 +205,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     clocks.start()
     total = 0.0
-    phase = [0.0, 0.0, 0.0]
+    phase = [0.0, 0.0, 0.0, 0.0]
     for _ in range(args.steps):
         flush.zero_()
         s0 = torch.cuda.Event(enable_timing=True)
@@ -216,8 +216,8 @@ def run_sdm(args, cfg, rank, world, local_rank):
         s1.synchronize()
         total += s0.elapsed_time(s1)
         for c in range(plan["chunks"]):
-            for j in range(3):
-                phase[j] += ev[4 * c + j].elapsed_time(ev[4 * c + j + 1])
+            for j in range(4):
+                phase[j] += ev[5 * c + j].elapsed_time(ev[5 * c + j + 1])
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -273,7 +273,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
     K = args.steps
     th = cfg.BH * cfg.T
     value = world * th * K / (t_max / 1e3)
-    names = ["score", "merge_plan", "recur"]
+    names = ["score", "merge", "plan", "recur"]
     shares = {n: phase[i] / max(1e-12, sum(phase)) for i, n in enumerate(names)}
     per = {n: phase[i] / K for i, n in enumerate(names)}
     dom = max(names, key=lambda n: per[n])
@@ -290,7 +290,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
     else:
         # CUDA-core kernels: float32 FMA peak = 148 SMs x 128 lanes x 2 x max clock
         fp32_peak = 148 * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
-        kname = "k_score_simt" if dom == "score" else "k_merge_plan"
+        kname = {"score": "k_score_simt", "merge": "k_merge", "plan": "k_plan"}[dom]
         roof = {"kernel": kname, "bound": "alu",
                 "achieved": (score_flops / (per[dom] / 1e3) / 1e12) if dom == "score" else None,
                 "peak": fp32_peak, "unit": "TFLOP/s"}

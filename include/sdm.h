@@ -142,8 +142,9 @@ SDM_API int sdm_recur(const void* v, const float* alpha, const float* beta, cons
 /*
  * sdm_forward that also records caller-created CUDA events (cudaEvent_t) on
  * `stream` at the boundaries of its kernel phases, for timing: for time chunk c
- * (see sdm_query_plan) events[4c+0] before scoring, [4c+1] after scoring,
- * [4c+2] after the merge/plan kernel, [4c+3] after the recurrence kernel.
+ * (see sdm_query_plan) events[5c+0] before scoring, [5c+1] after scoring,
+ * [5c+2] after the merge kernel, [5c+3] after the plan kernel, [5c+4] after
+ * the recurrence kernel.
  * Boundaries past n_events are not recorded.  Same results as sdm_forward.
  */
 SDM_API int sdm_forward_timed(const void* q, const void* k, const void* v, const float* alpha,
@@ -180,8 +181,9 @@ SDM_API int sdm_forward_noalloc(const void* q, const void* k, const void* v, con
  * How the library will run `dims` (host only, no GPU work).  Writes up to n
  * values into out: [0] tensor-core scoring (1) or CUDA-core scoring (0),
  * [1] survivor capacity per half-row, [2] steps per plan block P,
- * [3] slot parts per head G, [4] steps per time chunk, [5] number of chunks,
- * [6] kernel launches per sdm_forward call.  Returns SDM_OK or a dims error.
+ * [3] recurrence streams per head S, [4] steps per time chunk, [5] number of
+ * chunks, [6] kernel launches per sdm_forward call, [7] slot buckets per head.
+ * Returns SDM_OK or a dims error.
  */
 SDM_API int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n);
 

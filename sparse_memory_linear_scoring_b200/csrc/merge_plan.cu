@@ -18,15 +18,17 @@
 // The merge kernel writes the lists (slot, weight) of every step; the plan
 // kernel reads them back (or a caller's lists) and builds the recurrence plan.
 //
-// Plan (one CTA per (head, block of P steps)): the block's W+R entries per step
-// are grouped for the recurrence kernel.  Each slot belongs to one of G parts
-// (a hash of the slot); records are laid out part by part: the writes of slots
-// used once in the block, the reads of slots used once, then the slots used
-// several times, grouped by slot in time order (write before read within a
-// step).  A record is
-//   int4 {slot, (step_in_block << 1) | is_read, weight bits, chain length},
-// chain length = number of records of that slot in the block on its first
-// record, 0 on the others.
+// Plan (one CTA per (head, block of P steps)): the block's W+R entries per
+// step become records for the recurrence, ordered by (bucket, slot, entry).
+// A slot's bucket is a hash of the slot into the head's NB buckets, the same in
+// every block, and recurrence stream s owns buckets [s*mb, (s+1)*mb); so every
+// record of a slot, in every block, goes to the same stream, and within a
+// bucket a slot's records are adjacent and in time order (entry order puts a
+// step's write before its read).  A record is
+//   int4 {slot, (step_in_chunk << 1) | is_read, f1, f2}
+// with, for a write, f1 = alpha_t * (1 - c), f2 = c = beta_t * w_i (the update
+// is then M = f1 * M + f2 * v_t); for a read, f1 = u_r.  The per-(head, block)
+// bucket starts (NB + 1 of them) go to roff.
 #include "sdm_internal.cuh"
 
 namespace sdm {
@@ -67,27 +69,17 @@ __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
 
 size_t merge_smem_bytes(const Plan& p, int warps) { return merge_layout(p, warps).total; }
 
-// k_plan: the block's entries, a hash table of its slots (bit 31 marks a slot
-// used more than once), the multi-use list, and per-warp class counters.
+// k_plan: the block's sort keys (bucket, slot, entry) and the bucket counts /
+// starts and running positions.
 struct PlanLayout {
-  size_t ent_slot, ent_w, ent_key, hkey, mlist, cnt, off, misc, total;
-  int HS;
+  size_t key, cnt, total;
 };
 
 __host__ __device__ inline PlanLayout plan_layout(const Plan& p) {
   PlanLayout L;
-  L.HS = p2(2 * p.E);
-  const int nk = 3 * p.G;
-  const int nw = kMergeThreads / 32;
   size_t o = 0;
-  L.ent_slot = o; o = al16(o + size_t(p.E) * 4);
-  L.ent_w = o; o = al16(o + size_t(p.E) * 4);
-  L.ent_key = o; o = al16(o + size_t(p.E));
-  L.hkey = o; o = al16(o + size_t(L.HS) * 4);
-  L.mlist = o; o = al16(o + size_t(p2(p.E)) * 2);
-  L.cnt = o; o = al16(o + size_t(nw) * nk * 4);
-  L.off = o; o = al16(o + size_t(nw) * nk * 4);
-  L.misc = o; o = al16(o + size_t(2 * nk + 2 * kMaxParts + 8) * 4);
+  L.key = o; o = al16(o + size_t(p.E) * 8);
+  L.cnt = o; o = al16(o + size_t(2 * p.NB + 2) * 4);
   L.total = o;
   return L;
 }
@@ -442,26 +434,16 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   }
 }
 
-// One CTA per (head, block of P steps): group the block's list entries into
-// the recurrence plan (see the file header) and zero the block's rows of o.
-__global__ void __launch_bounds__(kMergeThreads)
+// One CTA per (head, block of P steps): sort the block's list entries into
+// records by (bucket, slot, entry) (see the file header) and zero the block's
+// rows of o.
+__global__ void __launch_bounds__(kPlanThreads)
 k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
   extern __shared__ __align__(16) unsigned char smem[];
   const PlanLayout L = plan_layout(p);
-  uint32_t* ent_slot = reinterpret_cast<uint32_t*>(smem + L.ent_slot);
-  float* ent_w = reinterpret_cast<float*>(smem + L.ent_w);
-  uint8_t* ent_key = smem + L.ent_key;
-  uint32_t* hkey = reinterpret_cast<uint32_t*>(smem + L.hkey);
-  uint16_t* mlist = reinterpret_cast<uint16_t*>(smem + L.mlist);
-  const int NK = 3 * p.G;                 // class keys: part * 3 + {single write, read, multi}
-  constexpr int NW = kMergeThreads / 32;
-  int* cnt = reinterpret_cast<int*>(smem + L.cnt);   // [NW][NK]
-  int* off = reinterpret_cast<int*>(smem + L.off);   // [NW][NK]
-  int* tot = reinterpret_cast<int*>(smem + L.misc);  // [NK] totals, then [NK] bases
-  int* kbase = tot + NK;
-  int* mbase = kbase + NK;                           // [G] start of a part's multis in mlist
-  int* misc = mbase + kMaxParts;                     // [0] n_multi
-
+  uint64_t* key = reinterpret_cast<uint64_t*>(smem + L.key);  // sorted by bucket
+  int* start = reinterpret_cast<int*>(smem + L.cnt);          // [NB + 1] counts, then starts
+  int* cur = start + p.NB + 1;                                 // [NB] running positions
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int WR = p.W + p.R;
@@ -469,188 +451,107 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
   if (s0 >= tlen) return;
   const int np = min(p.P, tlen - s0);
   const int nent = np * WR;
-  const uint32_t hmask = uint32_t(L.HS - 1);
-  constexpr uint32_t kMulti = 0x80000000u;
-
-  for (int i = tid; i < L.HS; i += blockDim.x) hkey[i] = kEmpty;
-  for (int i = tid; i < NW * NK; i += blockDim.x) cnt[i] = 0;
-  if (tid == 0) misc[0] = 0;
-  // entries, in step order, writes before reads
-  for (int e = tid; e < nent; e += blockDim.x) {
+  const size_t lrow0 = size_t(bh) * io.list_T + io.list_t0 + s0;  // list row of step s0
+  const size_t trow0 = size_t(bh) * p.T + t0 + s0;                 // time row of step s0
+  auto slot_of = [&](int e) -> int32_t {
     const int tl = e / WR, j = e - tl * WR;
-    const size_t row = size_t(bh) * io.list_T + io.list_t0 + s0 + tl;
-    int32_t s;
-    float w;
-    if (j < p.W) { s = io.iw[row * p.W + j]; w = io.ww[row * p.W + j]; }
-    else { s = io.ir[row * p.R + (j - p.W)]; w = io.wr[row * p.R + (j - p.W)]; }
-    if (s < 0 || (long long)s >= p.N) {
-      if (io.validate) dev_flag(st, SDM_DEV_BAD_INDEX, int(size_t(bh) * p.T + t0 + s0 + tl));
-      ent_slot[e] = kInvalid;
-    } else {
-      ent_slot[e] = uint32_t(s);
-    }
-    ent_w[e] = w;
-  }
+    return j < p.W ? io.iw[(lrow0 + tl) * p.W + j] : io.ir[(lrow0 + tl) * p.R + (j - p.W)];
+  };
+  auto in_range = [&](int32_t s) { return s >= 0 && (long long)s < p.N; };
+
+  for (int g = tid; g <= p.NB; g += blockDim.x) start[g] = 0;
   __syncthreads();
-  // hash table of the block's slots; a second sighting sets bit 31
   for (int e = tid; e < nent; e += blockDim.x) {
-    const uint32_t s = ent_slot[e];
-    if (s == kInvalid) continue;
-    uint32_t h = mix32(s) & hmask;
-    for (;;) {
-      const uint32_t old = atomicCAS(&hkey[h], kEmpty, s);
-      if (old == kEmpty) break;
-      if ((old & ~kMulti) == s) {
-        if (!(old & kMulti)) atomicOr(&hkey[h], kMulti);
-        break;
-      }
-      h = (h + 1) & hmask;
+    const int32_t s = slot_of(e);
+    if (!in_range(s)) {
+      if (io.validate) dev_flag(st, SDM_DEV_BAD_INDEX, int(trow0 + e / WR));
+      continue;
     }
-  }
-  __syncthreads();
-  // classify; count per (warp, key).  Warp w takes entries [w*chunk, (w+1)*chunk).
-  const int chunk = (nent + NW - 1) / NW;
-  const int e_lo = warp * chunk, e_hi = min(nent, e_lo + chunk);
-  for (int e = e_lo + lane; e < e_hi; e += 32) {
-    const uint32_t s = ent_slot[e];
-    uint8_t key = 0xff;
-    if (s != kInvalid) {
-      uint32_t h = mix32(s) & hmask;
-      while ((hkey[h] & ~kMulti) != s) h = (h + 1) & hmask;
-      const int part = slot_part(s, p.G);
-      int cls;
-      if (hkey[h] & kMulti) {
-        cls = 2;
-        mlist[atomicAdd(&misc[0], 1)] = uint16_t(e);
-      } else {
-        cls = (e % WR) < p.W ? 0 : 1;
-      }
-      key = uint8_t(part * 3 + cls);
-      atomicAdd(&cnt[warp * NK + key], 1);
-    }
-    ent_key[e] = key;
-  }
-  __syncthreads();
-  // totals per key, bases in part-major key order, per-warp offsets
-  for (int kk = tid; kk < NK; kk += blockDim.x) {
-    int t = 0;
-    for (int w = 0; w < NW; ++w) t += cnt[w * NK + kk];
-    tot[kk] = t;
+    atomicAdd(&start[slot_bucket(uint32_t(s), p.NB)], 1);
   }
   __syncthreads();
   if (warp == 0) {
-    // exclusive scans over the keys (and over the parts' multi counts), one warp
-    const int per = (NK + 31) / 32;
-    const int k0 = lane * per, k1 = min(NK, k0 + per);
-    int sa = 0, sm = 0;
-    for (int kk = k0; kk < k1; ++kk) {
-      sa += tot[kk];
-      if (kk % 3 == 2) sm += tot[kk];
-    }
-    int ia = sa, im = sm;
+    // exclusive scan of the bucket counts, one warp
+    const int per = (p.NB + 31) / 32;
+    const int g0 = min(p.NB, lane * per), g1 = min(p.NB, g0 + per);
+    int sum = 0;
+    for (int g = g0; g < g1; ++g) sum += start[g];
+    int inc = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, ia, o);
-      const int ym = __shfl_up_sync(0xffffffffu, im, o);
-      if (lane >= o) { ia += ya; im += ym; }
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
     }
-    int acc = ia - sa, macc = im - sm;
-    for (int kk = k0; kk < k1; ++kk) {
-      kbase[kk] = acc;
-      acc += tot[kk];
-      if (kk % 3 == 2) {
-        mbase[kk / 3] = macc;
-        macc += tot[kk];
-      }
+    int run = inc - sum;
+    for (int g = g0; g < g1; ++g) {
+      const int c = start[g];
+      start[g] = run;
+      cur[g] = run;
+      run += c;
     }
-    if (lane == 31) misc[1] = ia;
+    if (lane == 31) start[p.NB] = inc;
   }
   __syncthreads();
-  for (int kk = tid; kk < NK; kk += blockDim.x) {
-    int run = kbase[kk];
-    for (int w = 0; w < NW; ++w) {
-      off[w * NK + kk] = run;
-      run += cnt[w * NK + kk];
-    }
-  }
-  const int n_multi = misc[0];
-  // sort the multi-use entries by (part, slot, entry) -- ascending bitonic
-  {
-    const int S = n_multi > 1 ? p2(n_multi) : 1;
-    for (int i = n_multi + tid; i < S; i += blockDim.x) mlist[i] = 0xffff;
-    __syncthreads();
-    auto mkey = [&](uint16_t e) -> uint64_t {
-      if (e == 0xffff) return ~uint64_t(0);
-      const uint32_t s = ent_slot[e];
-      return (uint64_t(slot_part(s, p.G)) << 46) | (uint64_t(s) << 14) | uint64_t(e);
-    };
-    if (S <= 512) {
-      // few multi-use entries (the usual case): one warp sorts them
-      if (warp == 0) {
-        for (int size = 2; size <= S; size <<= 1) {
-          for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = lane; i < (S >> 1); i += 32) {
-              const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
-              const int hi = lo + stride;
-              const uint16_t x = mlist[lo], y = mlist[hi];
-              const uint64_t kx = mkey(x), ky = mkey(y);
-              const bool asc = (lo & size) == 0;
-              if (asc ? (kx > ky) : (kx < ky)) { mlist[lo] = y; mlist[hi] = x; }
-            }
-            __syncwarp();
-          }
-        }
-      }
-    } else for (int size = 2; size <= S; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < (S >> 1); i += blockDim.x) {
-          const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
-          const int hi = lo + stride;
-          const uint16_t x = mlist[lo], y = mlist[hi];
-          const uint64_t kx = mkey(x), ky = mkey(y);
-          const bool asc = (lo & size) == 0;
-          if (asc ? (kx > ky) : (kx < ky)) { mlist[lo] = y; mlist[hi] = x; }
-        }
-        __syncthreads();
-      }
-    }
+  int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (p.NB + 1);
+  for (int g = tid; g <= p.NB; g += blockDim.x) roff[g] = start[g];
+  for (int e = tid; e < nent; e += blockDim.x) {
+    const int32_t s = slot_of(e);
+    if (!in_range(s)) continue;
+    const int g = slot_bucket(uint32_t(s), p.NB);
+    const int pos = atomicAdd(&cur[g], 1);
+    key[pos] = (uint64_t(g) << (31 + kEntryBits)) | (uint64_t(uint32_t(s)) << kEntryBits) |
+               uint64_t(e);
   }
   __syncthreads();
+  // Each entry's record goes to its bucket's start plus its rank inside the
+  // bucket; its predecessor in that order tells whether a slot repeats within
+  // one step's list.
   int4* rec = io.rec + (size_t(bh) * p.nblk + blk) * p.E;
-  auto meta_of = [&](int e) -> int {
-    const int tl = e / WR;
-    return (tl << 1) | ((e - tl * WR) >= p.W ? 1 : 0);
-  };
-  // single-use entries: per-warp positions
-  for (int e = e_lo + lane; e < e_hi; e += 32) {
-    const uint8_t key = ent_key[e];
-    if (key == 0xff || key % 3 == 2) continue;
-    const int pos = atomicAdd(&off[warp * NK + key], 1);
-    rec[pos] = make_int4(int(ent_slot[e]), meta_of(e), __float_as_int(ent_w[e]), 1);
-  }
-  // multi-use entries: in sorted order, chains
-  for (int i = tid; i < n_multi; i += blockDim.x) {
-    const int e = mlist[i];
-    const uint32_t s = ent_slot[e];
-    const int part = slot_part(s, p.G);
-    const int pos = kbase[part * 3 + 2] + (i - mbase[part]);
-    int len = 0;
-    if (i == 0 || ent_slot[mlist[i - 1]] != s) {
-      int j = i + 1;
-      while (j < n_multi && ent_slot[mlist[j]] == s) ++j;
-      len = j - i;
-    } else if (meta_of(mlist[i - 1]) == meta_of(e)) {
-      dev_flag(st, SDM_DEV_BAD_LIST, int(size_t(bh) * p.T + t0 + s0 + e / WR));
+  const int total = start[p.NB];
+  constexpr uint64_t kEntryMask = (uint64_t(1) << kEntryBits) - 1;
+  for (int pos = tid; pos < total; pos += blockDim.x) {
+    const uint64_t x = key[pos];
+    const int g = int(x >> (31 + kEntryBits));
+    const uint32_t s = uint32_t(x >> kEntryBits) & 0x7fffffffu;
+    const int e = int(x & kEntryMask);
+    const int tl = e / WR, j = e - tl * WR;
+    const bool is_read = j >= p.W;
+    const float w = is_read ? io.wr[(lrow0 + tl) * p.R + (j - p.W)] : io.ww[(lrow0 + tl) * p.W + j];
+    float al = 0.f, be = 0.f;
+    if (!is_read) {
+      al = io.alpha[trow0 + tl];
+      be = io.beta[trow0 + tl];
     }
-    rec[pos] = make_int4(int(s), meta_of(e), __float_as_int(ent_w[e]), len);
+    const int b0 = start[g], n = start[g + 1] - b0;
+    int rank = 0;
+    uint64_t pred = 0;
+    for (int i = 0; i < n; ++i) {
+      const uint64_t y = key[b0 + i];
+      const bool lt = y < x;
+      rank += lt ? 1 : 0;
+      pred = (lt && y > pred) ? y : pred;
+    }
+    if (rank > 0 && (uint32_t(pred >> kEntryBits) & 0x7fffffffu) == s) {
+      const int e2 = int(pred & kEntryMask);
+      const int tl2 = e2 / WR;
+      if (tl2 == tl && ((e2 - tl2 * WR) >= p.W) == is_read)
+        dev_flag(st, SDM_DEV_BAD_LIST, int(trow0 + tl));
+    }
+    int4 r;
+    r.x = int(s);
+    r.y = ((s0 + tl) << 1) | (is_read ? 1 : 0);
+    if (is_read) {
+      r.z = __float_as_int(w);
+      r.w = 0;
+    } else {
+      const float c = be * w;
+      r.z = __float_as_int(al * (1.f - c));
+      r.w = __float_as_int(c);
+    }
+    rec[b0 + rank] = r;
   }
-  // per part g: single writes [3g, 3g+1), single reads [3g+1, 3g+2), multi-use
-  // chains [3g+2, 3g+3); entry 3G = end
-  int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (3 * p.G + 1);
-  for (int kk = tid; kk < NK; kk += blockDim.x) roff[kk] = kbase[kk];
-  if (tid == 0) roff[NK] = misc[1];
   // the recurrence adds every read into o with reductions: start from zero
-  float4* o4 = reinterpret_cast<float4*>(io.o + (size_t(bh) * p.T + t0 + s0) * p.dv);
+  float4* o4 = reinterpret_cast<float4*>(io.o + trow0 * p.dv);
   const int n4 = np * p.dv / 4;
   for (int i = tid; i < n4; i += blockDim.x) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -673,7 +574,7 @@ cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevSt
                                        int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((tlen + p.P - 1) / p.P, p.BH);
-  k_plan<<<grid, kMergeThreads, smem, s>>>(p, io, t0, tlen, st);
+  k_plan<<<grid, kPlanThreads, smem, s>>>(p, io, t0, tlen, st);
   return cudaGetLastError();
 }
 

@@ -8,20 +8,21 @@
 //           all other slots are untouched;
 //   item 4  o_t = sum_r u_r * M_t[r], read after step t's write.
 //
-// Work split.  Each (b,h) head is served by G CTAs; CTA g owns the slots whose
-// hash falls in part g, so no two CTAs ever touch the same row.  A CTA walks
-// the time blocks of the plan in order; inside a block its records are
-// independent except for slots used several times, whose records form one
-// chain handled in time order by a single thread group.  A slot row (d_v fp32)
-// is moved whole by L threads holding F = 4 or 8 floats each.  A block's
-// records come in three runs: writes of slots used once in the block, reads of
-// slots used once, and chains of slots used several times; the two single-use
-// runs are branch-free gathers (write: gate + delta + scatter; read: weight +
-// vector reduction into o, which the plan kernel zeroed).  The next block's
-// records, v rows and gates are prefetched with cp.async while a block runs.
-//
-// Between blocks a CTA barrier orders this CTA's row stores before its next
-// row loads; rows of other parts are never touched, so nothing else is needed.
+// Work split.  A head's slots are hashed into NB buckets, and each of the
+// head's S streams owns a fixed range of buckets: every record of a slot, in
+// every time block, belongs to one stream, so no two streams ever touch the
+// same row and a stream needs no barrier and no shared memory.  A stream is
+// one warp (LPR = 32 lanes, F = d_v / 32 floats of a row each) or, for
+// d_v < 32, a group of LPR = d_v lanes.  It walks the time blocks in order;
+// in each block its records are sorted by (bucket, slot, step, write before
+// read), so a slot's records are adjacent and in time order.  Records are
+// taken U at a time: every lane loads its share of the rows of the U records
+// at once (the first record of each slot run only), then the records are
+// applied in order -- a write is M = f1 * M + f2 * v_t (f1 = alpha (1 - c),
+// f2 = c, folded by the plan kernel), a read adds u * M to o_t with a vector
+// reduction (o was zeroed by the plan kernel) -- and each run's row is stored
+// once after its last write.  The next chunk's records and the next blocks'
+// segment bounds are loaded one step ahead.
 #include "sdm_internal.cuh"
 
 namespace sdm {
@@ -45,309 +46,392 @@ __device__ __forceinline__ void red_add4(float* ptr, float4 v) {
                : "memory");
 }
 
-// cp.async of n bytes (a multiple of 4) from global to shared memory, in 16-,
-// 8- or 4-byte pieces as the alignment of both ends allows.
-__device__ __forceinline__ void async_copy(void* dst, const void* src, int nbytes) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
-  const uintptr_t sa = reinterpret_cast<uintptr_t>(src);
-  const int al = int((sa | d | uintptr_t(nbytes)) & 15);
-  if (al == 0) {
-    for (int i = threadIdx.x * 16; i < nbytes; i += blockDim.x * 16)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + i), "l"(sa + i)
-                   : "memory");
-  } else if ((al & 7) == 0) {
-    for (int i = threadIdx.x * 8; i < nbytes; i += blockDim.x * 8)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d + i), "l"(sa + i)
-                   : "memory");
-  } else {
-    for (int i = threadIdx.x * 4; i < nbytes; i += blockDim.x * 4)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d + i), "l"(sa + i)
-                   : "memory");
-  }
-}
-__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void async_wait_prev() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
-
-template <typename Tv>
-__device__ __forceinline__ float4 v4_of(const Tv* row);
-template <>
-__device__ __forceinline__ float4 v4_of<float>(const float* row) {
-  return *reinterpret_cast<const float4*>(row);
-}
-template <>
-__device__ __forceinline__ float4 v4_of<__nv_bfloat16>(const __nv_bfloat16* row) {
-  const uint2 u = *reinterpret_cast<const uint2*>(row);
-  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-}
-
-// F consecutive floats of a staged v row as fp32
-template <typename Tv, int F>
-__device__ __forceinline__ void v_row(const Tv* row, float* out);
-template <>
-__device__ __forceinline__ void v_row<float, 4>(const float* row, float* out) {
-  const float4 a = *reinterpret_cast<const float4*>(row);
-  out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
-}
-template <>
-__device__ __forceinline__ void v_row<float, 8>(const float* row, float* out) {
-  const float4 a = reinterpret_cast<const float4*>(row)[0];
-  const float4 b = reinterpret_cast<const float4*>(row)[1];
-  out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
-  out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
-}
-__device__ __forceinline__ void bf16x2(uint32_t u, float* out) {
-  out[0] = __uint_as_float(u << 16);
-  out[1] = __uint_as_float(u & 0xffff0000u);
-}
-template <>
-__device__ __forceinline__ void v_row<__nv_bfloat16, 4>(const __nv_bfloat16* row, float* out) {
-  const uint2 u = *reinterpret_cast<const uint2*>(row);
-  bf16x2(u.x, out);
-  bf16x2(u.y, out + 2);
-}
-template <>
-__device__ __forceinline__ void v_row<__nv_bfloat16, 8>(const __nv_bfloat16* row, float* out) {
-  const uint4 u = *reinterpret_cast<const uint4*>(row);
-  bf16x2(u.x, out);
-  bf16x2(u.y, out + 2);
-  bf16x2(u.z, out + 4);
-  bf16x2(u.w, out + 6);
-}
-
 template <int F>
 __device__ __forceinline__ void ld_row(const float* ptr, float* m) {
-#pragma unroll
-  for (int j = 0; j < F / 4; ++j) {
-    const float4 x = ld_cg4(ptr + 4 * j);
-    m[4 * j] = x.x; m[4 * j + 1] = x.y; m[4 * j + 2] = x.z; m[4 * j + 3] = x.w;
+  if constexpr (F == 8) {
+    const float4 x = ld_cg4(ptr), y = ld_cg4(ptr + 4);
+    m[0] = x.x; m[1] = x.y; m[2] = x.z; m[3] = x.w;
+    m[4] = y.x; m[5] = y.y; m[6] = y.z; m[7] = y.w;
+  } else if constexpr (F == 4) {
+    const float4 x = ld_cg4(ptr);
+    m[0] = x.x; m[1] = x.y; m[2] = x.z; m[3] = x.w;
+  } else if constexpr (F == 2) {
+    float2 x;
+    asm volatile("ld.global.cg.v2.f32 {%0,%1}, [%2];" : "=f"(x.x), "=f"(x.y) : "l"(ptr));
+    m[0] = x.x; m[1] = x.y;
+  } else {
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(m[0]) : "l"(ptr));
   }
 }
 template <int F>
 __device__ __forceinline__ void st_row(float* ptr, const float* m) {
-#pragma unroll
-  for (int j = 0; j < F / 4; ++j)
-    st4(ptr + 4 * j, make_float4(m[4 * j], m[4 * j + 1], m[4 * j + 2], m[4 * j + 3]));
+  if constexpr (F == 8) {
+    st4(ptr, make_float4(m[0], m[1], m[2], m[3]));
+    st4(ptr + 4, make_float4(m[4], m[5], m[6], m[7]));
+  } else if constexpr (F == 4) {
+    st4(ptr, make_float4(m[0], m[1], m[2], m[3]));
+  } else if constexpr (F == 2) {
+    asm volatile("st.global.v2.f32 [%0], {%1,%2};" ::"l"(ptr), "f"(m[0]), "f"(m[1]) : "memory");
+  } else {
+    asm volatile("st.global.f32 [%0], %1;" ::"l"(ptr), "f"(m[0]) : "memory");
+  }
 }
 template <int F>
 __device__ __forceinline__ void red_row(float* ptr, const float* m, float u) {
-#pragma unroll
-  for (int j = 0; j < F / 4; ++j)
-    red_add4(ptr + 4 * j, make_float4(u * m[4 * j], u * m[4 * j + 1], u * m[4 * j + 2],
-                                      u * m[4 * j + 3]));
-}
-// M~ = alpha m;  M = (1 - c) M~ + c v,  c = beta w  (as alpha (1 - c) m + c v)
-template <int F>
-__device__ __forceinline__ void gate_delta(float* m, float alpha, float c, const float* vv) {
-  const float a = alpha * (1.f - c);
-#pragma unroll
-  for (int j = 0; j < F; ++j) m[j] = fmaf(a, m[j], c * vv[j]);
+  if constexpr (F == 8) {
+    red_add4(ptr, make_float4(u * m[0], u * m[1], u * m[2], u * m[3]));
+    red_add4(ptr + 4, make_float4(u * m[4], u * m[5], u * m[6], u * m[7]));
+  } else if constexpr (F == 4) {
+    red_add4(ptr, make_float4(u * m[0], u * m[1], u * m[2], u * m[3]));
+  } else if constexpr (F == 2) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1,%2};" ::"l"(ptr), "f"(u * m[0]), "f"(u * m[1])
+                 : "memory");
+  } else {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(ptr), "f"(u * m[0]) : "memory");
+  }
 }
 
-struct RecurLayout {
-  size_t roff, rec, v, ab, total;
+// F consecutive elements of a v row, raw (Vw 32-bit words), and as fp32
+template <typename Tv, int F>
+struct VRaw {
+  static constexpr int n = (sizeof(Tv) * F + 3) / 4;
+  uint32_t w[n];
+};
+template <typename Tv, int F>
+__device__ __forceinline__ void ld_v(const Tv* ptr, VRaw<Tv, F>& r) {
+  if constexpr (VRaw<Tv, F>::n == 8) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(ptr));
+    const uint4 y = __ldg(reinterpret_cast<const uint4*>(ptr) + 1);
+    r.w[0] = x.x; r.w[1] = x.y; r.w[2] = x.z; r.w[3] = x.w;
+    r.w[4] = y.x; r.w[5] = y.y; r.w[6] = y.z; r.w[7] = y.w;
+  } else if constexpr (VRaw<Tv, F>::n == 4) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(ptr));
+    r.w[0] = x.x; r.w[1] = x.y; r.w[2] = x.z; r.w[3] = x.w;
+  } else if constexpr (VRaw<Tv, F>::n == 2) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(ptr));
+    r.w[0] = x.x; r.w[1] = x.y;
+  } else if constexpr (sizeof(Tv) * F == 2) {
+    r.w[0] = __ldg(reinterpret_cast<const unsigned short*>(ptr));
+  } else {
+    r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(ptr));
+  }
+}
+template <typename Tv, int F>
+__device__ __forceinline__ float v_at(const VRaw<Tv, F>& r, int j) {
+  if constexpr (sizeof(Tv) == 4) {
+    return __uint_as_float(r.w[j]);
+  } else {
+    const uint32_t u = r.w[j >> 1];
+    return (j & 1) ? __uint_as_float(u & 0xffff0000u) : __uint_as_float(u << 16);
+  }
+}
+
+// shared-memory record reads that the compiler neither merges nor hoists, so
+// that a record's fields are live only where they are used
+__device__ __forceinline__ int2 lds2(const int4* ptr) {
+  int2 r;
+  asm volatile("ld.shared.v2.s32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(ptr))));
+  return r;
+}
+__device__ __forceinline__ int4 lds4(const int4* ptr) {
+  int4 r;
+  asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(ptr))));
+  return r;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// cp.async of NB bytes (4, 8, 16 or a multiple of 16) from global to shared
+template <int NB>
+__device__ __forceinline__ void cp_bytes(void* dst, const void* src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  if constexpr (NB >= 16) {
+#pragma unroll
+    for (int i = 0; i < NB / 16; ++i)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + 16 * i),
+                   "l"(static_cast<const char*>(src) + 16 * i)
+                   : "memory");
+  } else {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(d), "l"(src), "n"(NB)
+                 : "memory");
+  }
+}
+
+template <typename Tv, int LPR, int F>
+struct RecurSmem {
+  static constexpr int dv = LPR * F;
+  static constexpr int U = kRecurChunk;
+  static constexpr int kStreams = kRecurThreads / LPR;
+  // per stream: two chunks of records (the one applied, the one arriving),
+  // then the chunk's rows of M and of v
+  static constexpr size_t ring = size_t(2) * U * 16;
+  static constexpr size_t mrow = size_t(U) * dv * 4;
+  static constexpr size_t vrow = (size_t(U) * dv * sizeof(Tv) + 15) & ~size_t(15);
+  static constexpr size_t per_stream = ring + mrow + vrow;
+  static constexpr size_t total = per_stream * kStreams;
 };
 
-// Records of one (block, part) staged in shared memory; a part with more
-// records in a block reads the rest from global memory.
-constexpr int kRecStage = 512;
-
-__host__ __device__ inline RecurLayout recur_layout(const Plan& p) {
-  RecurLayout L;
-  const size_t vb = (p.dtype == SDM_DTYPE_F32 ? 4 : 2);
-  size_t o = 0;
-  L.roff = o; o += ((size_t(p.nblk) + 1) * 16 + 15) & ~size_t(15);
-  L.rec = o; o += size_t(2) * kRecStage * 16;
-  L.v = o; o += (size_t(2) * p.P * p.dv * vb + 15) & ~size_t(15);
-  L.ab = o; o += size_t(2) * 2 * p.P * 4;
-  L.total = o;
-  return L;
-}
-
-template <typename Tv, int F, int L>
-__global__ void __launch_bounds__(kRecurThreads, 2)
-k_recur(Plan p, const Tv* __restrict__ v, const float* __restrict__ alpha,
-        const float* __restrict__ beta, float* __restrict__ M, float* __restrict__ o,
-        const int4* __restrict__ rec, const int* __restrict__ roff, int t0, int tlen,
-        DevStatus* st) {
+template <typename Tv, int LPR, int F>
+__global__ void __launch_bounds__(kRecurThreads, kRecurWarps / 148 / (kRecurThreads / 32))
+k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restrict__ o,
+        const int4* __restrict__ rec, const int* __restrict__ roff, int t0, int tlen) {
+  using SM = RecurSmem<Tv, LPR, F>;
+  constexpr int dv = LPR * F;
+  constexpr int U = SM::U;
   extern __shared__ __align__(16) unsigned char smem[];
-  const RecurLayout Y = recur_layout(p);
-  constexpr int dv = F * L;
-  int* roff_s = reinterpret_cast<int*>(smem + Y.roff);   // [nb][4]
-  int4* rec_s = reinterpret_cast<int4*>(smem + Y.rec);   // [2][kRecStage]
-  Tv* v_s = reinterpret_cast<Tv*>(smem + Y.v);           // [2][P][dv]
-  float* ab_s = reinterpret_cast<float*>(smem + Y.ab);   // [2][alpha P | beta P]
-
-  const int part = blockIdx.x, bh = blockIdx.y;
-  constexpr int NG = kRecurThreads / L;
-  constexpr int kUnroll = kRecurUnroll * 4 / F;  // rows in flight per thread: 4*kRecurUnroll floats
-  const int grp = threadIdx.x / L, lg = threadIdx.x % L;
-  float* Mh = M + size_t(bh) * size_t(p.N) * dv + lg * F;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int stream = tid / LPR;
+  const int ls = threadIdx.x / LPR;  // stream within the CTA
+  const int sl = threadIdx.x % LPR;
+  unsigned char* mine = smem + size_t(ls) * SM::per_stream;
+  int4* ring = reinterpret_cast<int4*>(mine);                           // [2][U]
+  float* mrow = reinterpret_cast<float*>(mine + SM::ring) + sl * F;     // [U][dv], own part
+  Tv* vrow = reinterpret_cast<Tv*>(mine + SM::ring + SM::mrow) + sl * F;  // [U][dv], own part
+  const unsigned gmask =
+      LPR == 32 ? 0xffffffffu : (((1u << LPR) - 1u) << ((threadIdx.x & 31) / LPR * LPR));
+  const int bh = stream / p.S, s = stream - bh * p.S;
+  if (bh >= p.BH) return;  // whole lane groups leave together
   const int nb = (tlen + p.P - 1) / p.P;
+  const int g0 = s * p.mb, g1 = g0 + p.mb;
+  float* Mh = M + size_t(bh) * size_t(p.N) * dv + sl * F;
+  const size_t trow = size_t(bh) * p.T + t0;
+  const Tv* vh = v + trow * dv + sl * F;
+  float* oh = o + trow * dv + sl * F;
+  const int* rofh = roff + size_t(bh) * p.nblk * (p.NB + 1);
+  const int4* rech = rec + size_t(bh) * p.nblk * p.E;
 
-  // this part's [writes, reads, chains, end) record offsets in every block
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
-    const int* ro = roff + (size_t(bh) * p.nblk + b) * (3 * p.G + 1) + 3 * part;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) roff_s[4 * b + j] = __ldg(ro + j);
-  }
-  __syncthreads();
-
-  auto prefetch = [&](int b) {
-    const int buf = b & 1;
-    const int s0 = b * p.P;
-    const int np = min(p.P, tlen - s0);
-    const size_t trow = size_t(bh) * p.T + t0 + s0;
-    const size_t blk = size_t(bh) * p.nblk + b;
-    const int w0 = roff_s[4 * b];
-    const int nr = min(roff_s[4 * b + 3] - w0, kRecStage);
-    if (nr > 0) async_copy(rec_s + buf * kRecStage, rec + blk * p.E + w0, nr * 16);
-    async_copy(v_s + size_t(buf) * p.P * dv, v + trow * dv, int(np * dv * sizeof(Tv)));
-    async_copy(ab_s + buf * 2 * p.P, alpha + trow, np * 4);
-    async_copy(ab_s + buf * 2 * p.P + p.P, beta + trow, np * 4);
+  // Segment bounds of blocks [wb, wb + LPR) (lane j: block wb + j) and of the
+  // window after it.
+  int wb = 0, wlo, whi, nlo, nhi;
+  auto load_win = [&](int base, int& lo, int& hi) {
+    const int blk = base + sl;
+    lo = hi = 0;
+    if (blk < nb) {
+      const int* rr = rofh + size_t(blk) * (p.NB + 1);
+      lo = __ldg(rr + g0);
+      hi = __ldg(rr + g1);
+    }
   };
-
-  prefetch(0);
-  async_commit();
-  for (int b = 0; b < nb; ++b) {
-    if (b + 1 < nb) prefetch(b + 1);
-    async_commit();
-    async_wait_prev();
-    __syncthreads();
-    const int buf = b & 1;
-    const size_t trow = size_t(bh) * p.T + t0 + size_t(b) * p.P;
-    const int w0 = roff_s[4 * b];
-    const int nw = roff_s[4 * b + 1] - w0;   // single-use writes [0, nw)
-    const int nr = roff_s[4 * b + 2] - w0;   // single-use reads  [nw, nr)
-    const int ne = roff_s[4 * b + 3] - w0;   // chains            [nr, ne)
-    const int4* rg = rec + (size_t(bh) * p.nblk + b) * p.E + w0;
-    const int4* rs = rec_s + buf * kRecStage;
-    const Tv* vb = v_s + size_t(buf) * p.P * dv + lg * F;
-    const float* al_s = ab_s + buf * 2 * p.P;
-    const float* be_s = al_s + p.P;
-    float* ob = o + trow * dv + lg * F;
-    auto get_rec = [&](int i) -> int4 { return i < kRecStage ? rs[i] : __ldg(rg + i); };
-    auto slot_ok = [&](int s) -> bool {
-      if ((unsigned long long)(unsigned)s < (unsigned long long)p.N) return true;
-      if (lg == 0) dev_flag(st, SDM_DEV_BAD_INDEX, s);
-      return false;
-    };
-
-    // single-use writes: gather, gate, delta, scatter
-    for (int i0 = grp; i0 < nw; i0 += NG * kUnroll) {
-      int slot[kUnroll], meta[kUnroll];
-      float wt[kUnroll], m[kUnroll][F];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int i = i0 + u * NG;
-        slot[u] = -1;
-        if (i < nw) {
-          const int4 r = get_rec(i);
-          if (slot_ok(r.x)) { slot[u] = r.x; meta[u] = r.y; wt[u] = __int_as_float(r.z); }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (slot[u] >= 0) ld_row<F>(Mh + size_t(unsigned(slot[u])) * dv, m[u]);
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (slot[u] < 0) continue;
-        const int tl = meta[u] >> 1;
-        float vv[F];
-        v_row<Tv, F>(vb + tl * dv, vv);
-        gate_delta<F>(m[u], al_s[tl], be_s[tl] * wt[u], vv);
-        st_row<F>(Mh + size_t(unsigned(slot[u])) * dv, m[u]);
-      }
+  // bounds of block x, wb <= x < wb + 2 LPR (empty past the last block)
+  auto bounds = [&](int x, int& lo, int& hi) {
+    const int j = x - wb;
+    const int l0 = __shfl_sync(gmask, wlo, j & (LPR - 1), LPR);
+    const int h0 = __shfl_sync(gmask, whi, j & (LPR - 1), LPR);
+    const int l1 = __shfl_sync(gmask, nlo, j & (LPR - 1), LPR);
+    const int h1 = __shfl_sync(gmask, nhi, j & (LPR - 1), LPR);
+    lo = j < LPR ? l0 : l1;
+    hi = j < LPR ? h0 : h1;
+  };
+  // A chunk is up to U records: the rest of block blk's segment from pos, then
+  // the start of block blk+1's.  Lanes copy the records into the ring.
+  auto fetch_chunk = [&](int buf, int blk, int pos, int end, int npos, int nend) {
+    const int t1 = min(U, end - pos);
+    const int t2 = blk + 1 < nb ? min(U - t1, nend - npos) : 0;
+    for (int i = sl; i < t1 + t2; i += LPR) {
+      const int4* src = i < t1 ? rech + size_t(blk) * p.E + pos + i
+                               : rech + size_t(blk + 1) * p.E + npos + (i - t1);
+      cp_bytes<16>(&ring[buf * U + i], src);
     }
-    // single-use reads: gather, weight, reduce into o
-    for (int i0 = nw + grp; i0 < nr; i0 += NG * kUnroll) {
-      int slot[kUnroll], meta[kUnroll];
-      float wt[kUnroll], m[kUnroll][F];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int i = i0 + u * NG;
-        slot[u] = -1;
-        if (i < nr) {
-          const int4 r = get_rec(i);
-          if (slot_ok(r.x)) { slot[u] = r.x; meta[u] = r.y; wt[u] = __int_as_float(r.z); }
-        }
+    cp_async_commit();
+  };
+  load_win(0, wlo, whi);
+  load_win(LPR, nlo, nhi);
+  int b = 0, pos, end, npos, nend;
+  bounds(0, pos, end);
+  bounds(1, npos, nend);
+  int buf = 0;
+  fetch_chunk(0, 0, pos, end, npos, nend);
+  int pre_b = 0, pre_pos = pos;
+
+  while (b < nb) {
+    if (pos >= end) {
+      // next block; keep the bounds window two blocks ahead
+      ++b;
+      pos = npos;
+      end = nend;
+      if (b >= wb + LPR) {
+        wb += LPR;
+        wlo = nlo;
+        whi = nhi;
+        load_win(wb + LPR, nlo, nhi);
       }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (slot[u] >= 0) ld_row<F>(Mh + size_t(unsigned(slot[u])) * dv, m[u]);
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (slot[u] >= 0) red_row<F>(ob + size_t(meta[u] >> 1) * dv, m[u], wt[u]);
+      bounds(b + 1, npos, nend);
+      continue;
     }
-    // slots used several times in the block: one chain each, in time order
-    for (int i = nr + grp; i < ne; i += NG) {
-      const int4 r0 = get_rec(i);
-      if (r0.w <= 0 || !slot_ok(r0.x)) continue;
-      float m[F];
-      ld_row<F>(Mh + size_t(unsigned(r0.x)) * dv, m);
-      bool wrote = false;
-      for (int c = 0; c < r0.w; ++c) {
-        const int4 r = c == 0 ? r0 : get_rec(i + c);
-        const int tl = r.y >> 1;
-        const float w = __int_as_float(r.z);
-        if ((r.y & 1) == 0) {
-          float vv[F];
-          v_row<Tv, F>(vb + tl * dv, vv);
-          gate_delta<F>(m, al_s[tl], be_s[tl] * w, vv);
-          wrote = true;
+    if (pre_b != b || pre_pos != pos) {
+      cp_async_wait_all();
+      __syncwarp(gmask);
+      fetch_chunk(buf, b, pos, end, npos, nend);
+    }
+    cp_async_wait_all();
+    __syncwarp(gmask);
+    const int4* rs = ring + buf * U;
+    const int t1 = min(U, end - pos);
+    int t2 = b + 1 < nb ? min(U - t1, nend - npos) : 0;
+    if (t2 > 0) {
+      // a slot of block b+1 that block b's part of the chunk also holds would
+      // be loaded before that part stores it: end the chunk at the block edge
+      bool clash = false;
+      for (int i = t1 + sl; i < t1 + t2; i += LPR) {
+        const int si = lds2(&rs[i]).x;
+        for (int j = 0; j < t1; ++j) clash |= lds2(&rs[j]).x == si;
+      }
+      if (__any_sync(gmask, clash)) t2 = 0;
+    }
+    const int n = t1 + t2;
+    // the next chunk's position, and the prefetch of its records
+    int qb = b, qpos = pos + t1, qend = end, qnpos = npos, qnend = nend;
+    if (t2 > 0 || pos + t1 >= end) {
+      qb = b + 1;
+      qpos = npos + t2;
+      qend = nend;
+      bounds(b + 2, qnpos, qnend);
+    }
+    if (qb < nb && qpos < qend) {
+      fetch_chunk(buf ^ 1, qb, qpos, qend, qnpos, qnend);
+      pre_b = qb;
+      pre_pos = qpos;
+    } else {
+      pre_b = -1;
+    }
+    // gather into shared memory: the first record of every slot run copies
+    // the row; writes copy v_t.  Each lane copies and later reads only its own
+    // F columns, so its own wait makes them visible.
+    uint32_t head = 0, last = 0;  // per record: first / last of its slot run
+    {
+      int prev = -1;
+      for (int u = 0; u < n; ++u) {
+        const int2 sm = lds2(&rs[u]);  // slot, meta
+        if (u == 0 || u == t1 || sm.x != prev) {
+          head |= 1u << u;
+          if (u > 0) last |= 1u << (u - 1);
+          cp_bytes<F * 4>(mrow + u * dv, Mh + size_t(unsigned(sm.x)) * dv);
+        }
+        if (!(sm.y & 1)) {
+          if constexpr (F * sizeof(Tv) >= 4)
+            cp_bytes<F * sizeof(Tv)>(vrow + u * dv, vh + size_t(sm.y >> 1) * dv);
+          else
+            vrow[u * dv] = vh[size_t(sm.y >> 1) * dv];
+        }
+        prev = sm.x;
+      }
+      last |= 1u << (n - 1);
+      cp_async_commit();
+      cp_async_wait_all();
+    }
+    // apply in order; store each run's row after its last record
+    {
+      float cur[F];
+      bool dirty = false;
+      for (int u = 0; u < n; ++u) {
+        const int4 r = lds4(&rs[u]);
+        const float f1 = __int_as_float(r.z), f2 = __int_as_float(r.w);
+        if ((head >> u) & 1u) {
+#pragma unroll
+          for (int j = 0; j < F; ++j) cur[j] = mrow[u * dv + j];
+        }
+        if (!(r.y & 1)) {
+#pragma unroll
+          for (int j = 0; j < F; ++j) cur[j] = fmaf(f1, cur[j], f2 * to_f32(vrow[u * dv + j]));
+          dirty = true;
         } else {
-          red_row<F>(ob + size_t(tl) * dv, m, w);
+          red_row<F>(oh + size_t(r.y >> 1) * dv, cur, f1);
+        }
+        if ((last >> u) & 1u) {
+          if (dirty) st_row<F>(Mh + size_t(unsigned(r.x)) * dv, cur);
+          dirty = false;
         }
       }
-      if (wrote) st_row<F>(Mh + size_t(unsigned(r0.x)) * dv, m);
     }
-    __syncthreads();
+    // every lane has read this chunk's records before the ring slot is reused
+    __syncwarp(gmask);
+    buf ^= (pre_b >= 0) ? 1 : 0;
+    // advance
+    if (qb != b) {
+      b = qb;
+      pos = qpos;
+      end = qend;
+      npos = qnpos;
+      nend = qnend;
+      if (b >= wb + LPR) {
+        wb += LPR;
+        wlo = nlo;
+        whi = nhi;
+        load_win(wb + LPR, nlo, nhi);
+      }
+    } else {
+      pos = qpos;
+    }
   }
-  async_wait_prev();
+  cp_async_wait_all();
 }
 
-size_t recur_smem_bytes(const Plan& p) { return recur_layout(p).total; }
-
-template <typename Tv, int F, int L>
-static cudaError_t launch_recur_t(const Plan& p, const void* v, const float* alpha,
-                                  const float* beta, float* M, float* o, const int4* rec,
-                                  const int* roff, int t0, int tlen, DevStatus* st,
+template <typename Tv, int LPR, int F>
+static cudaError_t launch_recur_t(const Plan& p, const void* v, float* M, float* o,
+                                  const int4* rec, const int* roff, int t0, int tlen,
                                   cudaStream_t s) {
-  const size_t smem = recur_smem_bytes(p);
-  cudaError_t e = cudaFuncSetAttribute(k_recur<Tv, F, L>,
+  const size_t smem = RecurSmem<Tv, LPR, F>::total;
+  cudaError_t e = cudaFuncSetAttribute(k_recur<Tv, LPR, F>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(p.G, p.BH);
-  k_recur<Tv, F, L><<<grid, kRecurThreads, smem, s>>>(p, (const Tv*)v, alpha, beta, M, o, rec,
-                                                       roff, t0, tlen, st);
+  const long long threads = (long long)p.BH * p.S * LPR;
+  const int grid = int((threads + kRecurThreads - 1) / kRecurThreads);
+  k_recur<Tv, LPR, F><<<grid, kRecurThreads, smem, s>>>(p, (const Tv*)v, M, o, rec, roff, t0,
+                                                        tlen);
   return cudaGetLastError();
 }
 
-// A row of d_v floats is moved by L threads holding F = 4 or 8 floats each.
+// Floats per lane F for a row width: kRecurMaxF, kept within [d_v / 32, d_v / 4]
+// so that a row takes 4..32 lanes.
+constexpr int recur_floats_per_lane(int dv) {
+  return (kRecurMaxF < dv / 4 ? (kRecurMaxF > dv / 32 ? kRecurMaxF : dv / 32) : dv / 4) < 1
+             ? 1
+             : (kRecurMaxF < dv / 4 ? (kRecurMaxF > dv / 32 ? kRecurMaxF : dv / 32) : dv / 4);
+}
+
+int recur_lanes_per_row(int dv) { return dv / recur_floats_per_lane(dv); }
+
+template <typename Tv, int DV>
+static cudaError_t launch_recur_w(const Plan& p, const void* v, float* M, float* o,
+                                  const int4* rec, const int* roff, int t0, int tlen,
+                                  cudaStream_t s) {
+  constexpr int F = recur_floats_per_lane(DV);
+  return launch_recur_t<Tv, DV / F, F>(p, v, M, o, rec, roff, t0, tlen, s);
+}
+
 template <typename Tv>
-static cudaError_t launch_recur_dt(const Plan& p, const void* v, const float* alpha,
-                                   const float* beta, float* M, float* o, const int4* rec,
-                                   const int* roff, int t0, int tlen, DevStatus* st,
+static cudaError_t launch_recur_dt(const Plan& p, const void* v, float* M, float* o,
+                                   const int4* rec, const int* roff, int t0, int tlen,
                                    cudaStream_t s) {
   switch (p.dv) {
-    case 4: return launch_recur_t<Tv, 4, 1>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
-    case 8: return launch_recur_t<Tv, 4, 2>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
-    case 16: return launch_recur_t<Tv, 4, 4>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
-    case 32: return launch_recur_t<Tv, 8, 4>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
-    case 64: return launch_recur_t<Tv, 8, 8>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
-    case 128: return launch_recur_t<Tv, 8, 16>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
+    case 4: return launch_recur_w<Tv, 4>(p, v, M, o, rec, roff, t0, tlen, s);
+    case 8: return launch_recur_w<Tv, 8>(p, v, M, o, rec, roff, t0, tlen, s);
+    case 16: return launch_recur_w<Tv, 16>(p, v, M, o, rec, roff, t0, tlen, s);
+    case 32: return launch_recur_w<Tv, 32>(p, v, M, o, rec, roff, t0, tlen, s);
+    case 64: return launch_recur_w<Tv, 64>(p, v, M, o, rec, roff, t0, tlen, s);
+    case 128: return launch_recur_w<Tv, 128>(p, v, M, o, rec, roff, t0, tlen, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_recur(const Plan& p, const void* v, const float* alpha, const float* beta,
-                         float* M, float* o, const int4* rec, const int* roff, int t0, int tlen,
-                         DevStatus* st, cudaStream_t s) {
+cudaError_t launch_recur(const Plan& p, const void* v, float* M, float* o, const int4* rec,
+                         const int* roff, int t0, int tlen, cudaStream_t s) {
   if (p.dtype == SDM_DTYPE_F32)
-    return launch_recur_dt<float>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
-  return launch_recur_dt<__nv_bfloat16>(p, v, alpha, beta, M, o, rec, roff, t0, tlen, st, s);
+    return launch_recur_dt<float>(p, v, M, o, rec, roff, t0, tlen, s);
+  return launch_recur_dt<__nv_bfloat16>(p, v, M, o, rec, roff, t0, tlen, s);
 }
 
 }  // namespace sdm

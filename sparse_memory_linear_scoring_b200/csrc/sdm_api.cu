@@ -8,7 +8,7 @@
 //      on CUDA cores);
 //   2. merge: top-W / top-R lists with softmax weights (into the workspace, or
 //      the caller's lists for sdm_select);
-//   3. plan: the lists grouped into the recurrence's per-part records;
+//   3. plan: the lists sorted into the recurrence's per-stream records;
 //   4. recur: the gated delta writes and the reads, in time order.
 #include <limits.h>
 #include <stdint.h>
@@ -21,7 +21,7 @@ namespace sdm {
 size_t score_simt_smem(const Plan& p);
 size_t merge_smem_bytes(const Plan& p, int warps);
 size_t plan_smem_bytes(const Plan& p);
-size_t recur_smem_bytes(const Plan& p);
+int recur_lanes_per_row(int dv);
 size_t score_tc_smem(const Plan& p);
 int score_tc_capacity(const sdm_dims* d);
 
@@ -75,22 +75,28 @@ int make_plan(const sdm_dims* d, Plan* p) {
   if (p->ncW < p->W || p->ncR < p->R) return SDM_ERR_UNSUPPORTED;
   int P = kMaxBlockEntries / (p->W + p->R);
   if (P > 1024) P = 1024;
-  // the recurrence stages v (double-buffered) and an fp32 accumulator per step
-  const int vbytes = p->dtype == SDM_DTYPE_F32 ? 4 : 2;
-  const int p_smem = int((96 * 1024) / (p->dv * (2 * vbytes + 4)));
-  if (P > p_smem) P = p_smem;
   if (p->T > 0 && P > p->T) P = p->T;
   if (P < 1) P = 1;
   p->P = P;
   p->E = P * (p->W + p->R);
-  int G = (kTargetCtas + p->BH - 1) / p->BH;
-  if (G > kMaxParts) G = kMaxParts;
-  if (G < 1) G = 1;
-  p->G = G;
+  // recurrence streams per head: fill the target warp count (a warp holds
+  // 32 / LPR streams), keeping at least kStreamMin records per stream and block
+  {
+    const long long per_warp = 32 / recur_lanes_per_row(p->dv);
+    long long S = (kRecurWarps * per_warp + p->BH - 1) / p->BH;
+    const long long smax = p->E / kStreamMin > 1 ? p->E / kStreamMin : 1;
+    if (S > smax) S = smax;
+    if (S < 1) S = 1;
+    p->S = int(S);
+    long long mb = (p->E / kBucketTarget + S - 1) / S;
+    if (mb < 1) mb = 1;
+    p->mb = int(mb);
+    p->NB = int(S * mb);
+  }
   // time chunk: bounded workspace
   const size_t per_step = size_t(p->BH) * (4 * 4 + size_t(4) * p->C * 8 + 4 * 4 +
                                            size_t(p->W + p->R) * (16 + 8)) +
-                          (size_t(p->BH) * (3 * p->G + 1) * 4 + size_t(P) - 1) / size_t(P);
+                          (size_t(p->BH) * (p->NB + 1) * 4 + size_t(P) - 1) / size_t(P);
   const long long Tround = ((long long)(p->T > 0 ? p->T : 1) + P - 1) / P * P;
   long long Tc = (long long)(kChunkBudget / per_step) / P * P;
   if (Tc < P) Tc = P;
@@ -100,7 +106,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
   p->nblk = int((Tc + P - 1) / P);
   p->merge_smem = merge_smem_bytes(*p, kMergeWarps);
   p->plan_smem = plan_smem_bytes(*p);
-  p->recur_smem = recur_smem_bytes(*p);
+  p->recur_smem = 0;
   p->score_smem = p->tc ? score_tc_smem(*p) : score_simt_smem(*p);
   if (p->merge_smem > kMaxSmem || p->plan_smem > kMaxSmem || p->recur_smem > kMaxSmem ||
       p->score_smem > kMaxSmem)
@@ -113,7 +119,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
   p->off_redo = o; o = align256(o + nhr * 4);
   p->off_lists = o; o = align256(o + size_t(p->BH) * p->Tc * (p->W + p->R) * 8);
   p->off_rec = o; o = align256(o + size_t(p->BH) * p->nblk * p->E * 16);
-  p->off_roff = o; o = align256(o + size_t(p->BH) * p->nblk * (3 * p->G + 1) * 4);
+  p->off_roff = o; o = align256(o + size_t(p->BH) * p->nblk * (p->NB + 1) * 4);
   p->total = o;
   return SDM_OK;
 }
@@ -240,22 +246,24 @@ static int forward_impl(const void* q, const void* k, const void* v, const float
   pio.list_T = p.Tc;
   pio.list_t0 = 0;
   pio.validate = 0;
+  pio.alpha = alpha;
+  pio.beta = beta;
   pio.rec = c.rec;
   pio.roff = c.roff;
   pio.o = o_out;
   for (int ch = 0; ch < p.nchunks; ++ch) {
     const int t0 = ch * p.Tc;
     const int tlen = (p.T - t0 < p.Tc) ? p.T - t0 : p.Tc;
-    if (!mark(4 * ch)) return SDM_ERR_CUDA;
+    if (!mark(5 * ch)) return SDM_ERR_CUDA;
     if (score_chunk(p, c, q, k, C1, C2, t0, tlen, s) != cudaSuccess) return SDM_ERR_CUDA;
-    if (!mark(4 * ch + 1)) return SDM_ERR_CUDA;
+    if (!mark(5 * ch + 1)) return SDM_ERR_CUDA;
     if (launch_merge(p, mio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
+    if (!mark(5 * ch + 2)) return SDM_ERR_CUDA;
     if (launch_plan(p, pio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
-    if (!mark(4 * ch + 2)) return SDM_ERR_CUDA;
-    if (launch_recur(p, v, alpha, beta, M_inout, o_out, c.rec, c.roff, t0, tlen, c.st, s) !=
-        cudaSuccess)
+    if (!mark(5 * ch + 3)) return SDM_ERR_CUDA;
+    if (launch_recur(p, v, M_inout, o_out, c.rec, c.roff, t0, tlen, s) != cudaSuccess)
       return SDM_ERR_CUDA;
-    if (!mark(4 * ch + 3)) return SDM_ERR_CUDA;
+    if (!mark(5 * ch + 4)) return SDM_ERR_CUDA;
   }
   return SDM_OK;
 }
@@ -282,8 +290,9 @@ extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
   const int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
   const int64_t per_chunk = (p.tc ? 3 : 1) + 3;
-  const int64_t vals[7] = {p.tc, p.C, p.P, p.G, p.Tc, p.nchunks, 1 + per_chunk * p.nchunks};
-  for (int i = 0; i < n && i < 7; ++i) out[i] = vals[i];
+  const int64_t vals[8] = {p.tc, p.C, p.P, p.S, p.Tc, p.nchunks, 1 + per_chunk * p.nchunks,
+                           p.NB};
+  for (int i = 0; i < n && i < 8; ++i) out[i] = vals[i];
   return SDM_OK;
 }
 
@@ -336,6 +345,8 @@ extern "C" int sdm_recur(const void* v, const float* alpha, const float* beta,
   pio.iw = idx_w; pio.ww = w_w; pio.ir = idx_r; pio.wr = w_r;
   pio.list_T = p.T;
   pio.validate = 1;
+  pio.alpha = alpha;
+  pio.beta = beta;
   pio.rec = c.rec;
   pio.roff = c.roff;
   pio.o = o_out;
@@ -344,8 +355,7 @@ extern "C" int sdm_recur(const void* v, const float* alpha, const float* beta,
     const int tlen = (p.T - t0 < p.Tc) ? p.T - t0 : p.Tc;
     pio.list_t0 = t0;
     if (launch_plan(p, pio, t0, tlen, c.st, s) != cudaSuccess) return SDM_ERR_CUDA;
-    if (launch_recur(p, v, alpha, beta, M_inout, o_out, c.rec, c.roff, t0, tlen, c.st, s) !=
-        cudaSuccess)
+    if (launch_recur(p, v, M_inout, o_out, c.rec, c.roff, t0, tlen, s) != cudaSuccess)
       return SDM_ERR_CUDA;
   }
   return SDM_OK;

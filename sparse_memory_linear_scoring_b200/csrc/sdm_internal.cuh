@@ -3,8 +3,8 @@
 // The forward pass is split into three kernel families, launched per time
 // chunk on the caller's stream:
 //   1. scoring + per-half candidate lists   (score_simt.cu, score_tc.cu)
-//   2. merge of the two halves into the top-W / top-R lists, softmax weights,
-//      and the write/read plan of the recurrence           (merge_plan.cu)
+//   2. merge of the two halves into the top-W / top-R lists and softmax
+//      weights, then the write/read plan of the recurrence (merge_plan.cu)
 //   3. the gated delta recurrence over the slot table     (recur.cu)
 #pragma once
 
@@ -18,24 +18,28 @@ namespace sdm {
 
 // Fixed launch targets (depend on nothing but the problem sizes, so the
 // workspace size is a function of the dims alone).
-#ifndef SDM_TARGET_CTAS
-#define SDM_TARGET_CTAS 296
+#ifndef SDM_RECUR_WARPS
+#define SDM_RECUR_WARPS 2368  // recurrence warps aimed for: 148 SMs x 16 resident warps
 #endif
-#ifndef SDM_RECUR_THREADS
-#define SDM_RECUR_THREADS 256
+#ifndef SDM_RECUR_CHUNK
+#define SDM_RECUR_CHUNK 8  // records of a recurrence stream whose rows are in flight at once
 #endif
-#ifndef SDM_RECUR_UNROLL
-#define SDM_RECUR_UNROLL 8
+#ifndef SDM_RECUR_MAX_F
+#define SDM_RECUR_MAX_F 8  // floats of a row per lane, at most
 #endif
-constexpr int kTargetCtas = SDM_TARGET_CTAS;  // recurrence CTAs aimed for (2 x 148 SMs)
-constexpr int kMaxParts = 64;           // slot parts per head in the recurrence
+constexpr int kRecurMaxF = SDM_RECUR_MAX_F;
+constexpr int kRecurWarps = SDM_RECUR_WARPS;
+constexpr int kRecurChunk = SDM_RECUR_CHUNK;
+constexpr int kRecurThreads = 256;
 constexpr int kMaxBlockEntries = 8192;  // list entries per (head, block) in a plan
+constexpr int kEntryBits = 13;          // entry index within a block: < 2^13
+static_assert(kMaxBlockEntries <= (1 << kEntryBits), "entry index must fit its key field");
+constexpr int kBucketTarget = 16;       // mean plan records per bucket aimed for
+constexpr int kStreamMin = 8;           // mean records per stream and block, at least
 constexpr size_t kChunkBudget = size_t(1) << 30;  // workspace bytes per time chunk
-constexpr int kMergeThreads = 512;     // plan kernel
+constexpr int kPlanThreads = 256;
 constexpr int kMergeWarps = 8;          // merge kernel: warps per CTA
 constexpr int kMergeSteps = 16;         // merge kernel: steps per CTA
-constexpr int kRecurThreads = SDM_RECUR_THREADS;
-constexpr int kRecurUnroll = SDM_RECUR_UNROLL;
 
 // Everything the kernels need to know about one call.
 struct Plan {
@@ -49,7 +53,9 @@ struct Plan {
   int P;       // steps per plan block
   int nblk;    // plan blocks per chunk
   int E;       // list entries per plan block = P * (W + R)
-  int G;       // slot parts per head
+  int S;       // recurrence streams per head (one warp, or a lane group for d_v < 32)
+  int NB;      // slot buckets per head = S * mb; stream s owns buckets [s*mb, (s+1)*mb)
+  int mb;
   int ncW, nfW, ncR, nfR;  // staircase / frontier sizes of the merge
   size_t merge_smem, plan_smem, recur_smem, score_smem;
   // workspace byte offsets
@@ -89,9 +95,9 @@ __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   x ^= x >> 16;
   return x;
 }
-// Which part (recurrence CTA) of a head owns a slot.
-__device__ __forceinline__ int slot_part(uint32_t slot, int G) {
-  return int(mix32(slot ^ 0x9e3779b9u) % uint32_t(G));
+// Which of a head's NB buckets holds a slot (multiply-shift of a hash).
+__device__ __forceinline__ int slot_bucket(uint32_t slot, int NB) {
+  return int((uint64_t(mix32(slot ^ 0x9e3779b9u)) * uint64_t(uint32_t(NB))) >> 32);
 }
 
 __device__ __forceinline__ void dev_flag(DevStatus* st, int bits, int info) {
@@ -155,7 +161,8 @@ cudaError_t launch_merge(const Plan& p, const MergeIO& io, int t0, int tlen, Dev
 struct PlanIO {
   const int32_t* iw; const float* ww; const int32_t* ir; const float* wr;
   int list_T, list_t0;
-  int validate;  // flag out-of-range slots (caller lists)
+  int validate;  // flag out-of-range slots and repeated slots (caller lists)
+  const float* alpha; const float* beta;
   int4* rec;
   int* roff;
   float* o;
@@ -163,8 +170,7 @@ struct PlanIO {
 cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevStatus* st,
                         cudaStream_t s);
 
-cudaError_t launch_recur(const Plan& p, const void* v, const float* alpha, const float* beta,
-                         float* M, float* o, const int4* rec, const int* roff, int t0, int tlen,
-                         DevStatus* st, cudaStream_t s);
+cudaError_t launch_recur(const Plan& p, const void* v, float* M, float* o, const int4* rec,
+                         const int* roff, int t0, int tlen, cudaStream_t s);
 
 }  // namespace sdm

@@ -129,8 +129,8 @@ def _dims_of(q: torch.Tensor, v: torch.Tensor, C1: torch.Tensor, topk: int, W: i
     return make_dims(B, H, T, d_qk, v.shape[-1], C1.shape[1], topk, W, R, q.dtype)
 
 
-PLAN_FIELDS = ("tensor_core_scoring", "survivor_capacity", "block_steps", "parts_per_head",
-               "chunk_steps", "chunks", "launches_per_call")
+PLAN_FIELDS = ("tensor_core_scoring", "survivor_capacity", "block_steps", "streams_per_head",
+               "chunk_steps", "chunks", "launches_per_call", "buckets_per_head")
 
 
 def query_plan(dims: Dims) -> Dict[str, int]:
