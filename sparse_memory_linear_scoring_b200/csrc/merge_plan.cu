@@ -453,21 +453,36 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
   const int nent = np * WR;
   const size_t lrow0 = size_t(bh) * io.list_T + io.list_t0 + s0;  // list row of step s0
   const size_t trow0 = size_t(bh) * p.T + t0 + s0;                 // time row of step s0
+  // e / WR for e < 2^13 by a multiply-high (exact in that range)
+  const uint32_t magic = 0xffffffffu / uint32_t(WR) + 1u;
+  auto step_of = [&](int e) { return int(__umulhi(uint32_t(e), magic)); };
   auto slot_of = [&](int e) -> int32_t {
-    const int tl = e / WR, j = e - tl * WR;
+    const int tl = step_of(e), j = e - tl * WR;
     return j < p.W ? io.iw[(lrow0 + tl) * p.W + j] : io.ir[(lrow0 + tl) * p.R + (j - p.W)];
   };
   auto in_range = [&](int32_t s) { return s >= 0 && (long long)s < p.N; };
+  constexpr int kB = 8;  // entries per thread whose loads are in flight together
+  const int stride = blockDim.x;
 
-  for (int g = tid; g <= p.NB; g += blockDim.x) start[g] = 0;
+  for (int g = tid; g <= p.NB; g += stride) start[g] = 0;
   __syncthreads();
-  for (int e = tid; e < nent; e += blockDim.x) {
-    const int32_t s = slot_of(e);
-    if (!in_range(s)) {
-      if (io.validate) dev_flag(st, SDM_DEV_BAD_INDEX, int(trow0 + e / WR));
-      continue;
+  for (int e0 = tid; e0 < nent; e0 += stride * kB) {
+    int32_t sv[kB];
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int e = e0 + i * stride;
+      sv[i] = e < nent ? slot_of(e) : 0;
     }
-    atomicAdd(&start[slot_bucket(uint32_t(s), p.NB)], 1);
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int e = e0 + i * stride;
+      if (e >= nent) break;
+      if (!in_range(sv[i])) {
+        if (io.validate) dev_flag(st, SDM_DEV_BAD_INDEX, int(trow0 + step_of(e)));
+        continue;
+      }
+      atomicAdd(&start[slot_bucket(uint32_t(sv[i]), p.NB)], 1);
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -493,14 +508,24 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
   }
   __syncthreads();
   int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (p.NB + 1);
-  for (int g = tid; g <= p.NB; g += blockDim.x) roff[g] = start[g];
-  for (int e = tid; e < nent; e += blockDim.x) {
-    const int32_t s = slot_of(e);
-    if (!in_range(s)) continue;
-    const int g = slot_bucket(uint32_t(s), p.NB);
-    const int pos = atomicAdd(&cur[g], 1);
-    key[pos] = (uint64_t(g) << (31 + kEntryBits)) | (uint64_t(uint32_t(s)) << kEntryBits) |
-               uint64_t(e);
+  for (int g = tid; g <= p.NB; g += stride) roff[g] = start[g];
+  for (int e0 = tid; e0 < nent; e0 += stride * kB) {
+    int32_t sv[kB];
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int e = e0 + i * stride;
+      sv[i] = e < nent ? slot_of(e) : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int e = e0 + i * stride;
+      if (e >= nent) break;
+      if (!in_range(sv[i])) continue;
+      const int g = slot_bucket(uint32_t(sv[i]), p.NB);
+      const int pos = atomicAdd(&cur[g], 1);
+      key[pos] = (uint64_t(g) << (31 + kEntryBits)) | (uint64_t(uint32_t(sv[i])) << kEntryBits) |
+                 uint64_t(e);
+    }
   }
   __syncthreads();
   // Each entry's record goes to its bucket's start plus its rank inside the
@@ -509,51 +534,69 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
   int4* rec = io.rec + (size_t(bh) * p.nblk + blk) * p.E;
   const int total = start[p.NB];
   constexpr uint64_t kEntryMask = (uint64_t(1) << kEntryBits) - 1;
-  for (int pos = tid; pos < total; pos += blockDim.x) {
-    const uint64_t x = key[pos];
-    const int g = int(x >> (31 + kEntryBits));
-    const uint32_t s = uint32_t(x >> kEntryBits) & 0x7fffffffu;
-    const int e = int(x & kEntryMask);
-    const int tl = e / WR, j = e - tl * WR;
-    const bool is_read = j >= p.W;
-    const float w = is_read ? io.wr[(lrow0 + tl) * p.R + (j - p.W)] : io.ww[(lrow0 + tl) * p.W + j];
-    float al = 0.f, be = 0.f;
-    if (!is_read) {
-      al = io.alpha[trow0 + tl];
-      be = io.beta[trow0 + tl];
+  constexpr int kR = 4;
+  for (int p0 = tid; p0 < total; p0 += stride * kR) {
+    uint64_t x[kR];
+    float w[kR], al[kR], be[kR];
+#pragma unroll
+    for (int i = 0; i < kR; ++i) {
+      const int pos = p0 + i * stride;
+      x[i] = pos < total ? key[pos] : 0;
+      const int e = int(x[i] & kEntryMask);
+      const int tl = step_of(e), j = e - tl * WR;
+      w[i] = al[i] = be[i] = 0.f;
+      if (pos < total) {
+        if (j >= p.W) {
+          w[i] = io.wr[(lrow0 + tl) * p.R + (j - p.W)];
+        } else {
+          w[i] = io.ww[(lrow0 + tl) * p.W + j];
+          al[i] = io.alpha[trow0 + tl];
+          be[i] = io.beta[trow0 + tl];
+        }
+      }
     }
-    const int b0 = start[g], n = start[g + 1] - b0;
-    int rank = 0;
-    uint64_t pred = 0;
-    for (int i = 0; i < n; ++i) {
-      const uint64_t y = key[b0 + i];
-      const bool lt = y < x;
-      rank += lt ? 1 : 0;
-      pred = (lt && y > pred) ? y : pred;
+#pragma unroll
+    for (int i = 0; i < kR; ++i) {
+      const int pos = p0 + i * stride;
+      if (pos >= total) break;
+      const int g = int(x[i] >> (31 + kEntryBits));
+      const uint32_t s = uint32_t(x[i] >> kEntryBits) & 0x7fffffffu;
+      const int e = int(x[i] & kEntryMask);
+      const int tl = step_of(e), j = e - tl * WR;
+      const bool is_read = j >= p.W;
+      const int b0 = start[g], n = start[g + 1] - b0;
+      int rank = 0;
+      uint64_t pred = 0;
+      for (int q = 0; q < n; ++q) {
+        const uint64_t y = key[b0 + q];
+        const bool lt = y < x[i];
+        rank += lt ? 1 : 0;
+        pred = (lt && y > pred) ? y : pred;
+      }
+      if (rank > 0 && (uint32_t(pred >> kEntryBits) & 0x7fffffffu) == s) {
+        const int e2 = int(pred & kEntryMask);
+        const int tl2 = step_of(e2);
+        if (tl2 == tl && ((e2 - tl2 * WR) >= p.W) == is_read)
+          dev_flag(st, SDM_DEV_BAD_LIST, int(trow0 + tl));
+      }
+      int4 r;
+      r.x = int(s);
+      r.y = ((s0 + tl) << 1) | (is_read ? 1 : 0);
+      if (is_read) {
+        r.z = __float_as_int(w[i]);
+        r.w = 0;
+      } else {
+        const float c = be[i] * w[i];
+        r.z = __float_as_int(al[i] * (1.f - c));
+        r.w = __float_as_int(c);
+      }
+      rec[b0 + rank] = r;
     }
-    if (rank > 0 && (uint32_t(pred >> kEntryBits) & 0x7fffffffu) == s) {
-      const int e2 = int(pred & kEntryMask);
-      const int tl2 = e2 / WR;
-      if (tl2 == tl && ((e2 - tl2 * WR) >= p.W) == is_read)
-        dev_flag(st, SDM_DEV_BAD_LIST, int(trow0 + tl));
-    }
-    int4 r;
-    r.x = int(s);
-    r.y = ((s0 + tl) << 1) | (is_read ? 1 : 0);
-    if (is_read) {
-      r.z = __float_as_int(w);
-      r.w = 0;
-    } else {
-      const float c = be * w;
-      r.z = __float_as_int(al * (1.f - c));
-      r.w = __float_as_int(c);
-    }
-    rec[b0 + rank] = r;
   }
   // the recurrence adds every read into o with reductions: start from zero
   float4* o4 = reinterpret_cast<float4*>(io.o + trow0 * p.dv);
   const int n4 = np * p.dv / 4;
-  for (int i = tid; i < n4; i += blockDim.x) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = tid; i < n4; i += stride) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 cudaError_t launch_merge(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,

@@ -313,7 +313,9 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
     uint32_t head = 0, last = 0;  // per record: first / last of its slot run
     {
       int prev = -1;
-      for (int u = 0; u < n; ++u) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (u >= n) break;
         const int2 sm = lds2(&rs[u]);  // slot, meta
         if (u == 0 || u == t1 || sm.x != prev) {
           head |= 1u << u;
@@ -336,7 +338,9 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
     {
       float cur[F];
       bool dirty = false;
-      for (int u = 0; u < n; ++u) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (u >= n) break;
         const int4 r = lds4(&rs[u]);
         const float f1 = __int_as_float(r.z), f2 = __int_as_float(r.w);
         if ((head >> u) & 1u) {

@@ -35,7 +35,7 @@ constexpr int kMaxBlockEntries = 8192;  // list entries per (head, block) in a p
 constexpr int kEntryBits = 13;          // entry index within a block: < 2^13
 static_assert(kMaxBlockEntries <= (1 << kEntryBits), "entry index must fit its key field");
 constexpr int kBucketTarget = 16;       // mean plan records per bucket aimed for
-constexpr int kStreamMin = 8;           // mean records per stream and block, at least
+constexpr int kStreamMin = 4;           // mean records per stream and block, at least
 constexpr size_t kChunkBudget = size_t(1) << 30;  // workspace bytes per time chunk
 constexpr int kPlanThreads = 256;
 constexpr int kMergeWarps = 8;          // merge kernel: warps per CTA
