@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--probe-rows", action="store_true",
+                    help="measure the HBM ceiling of random 256-byte row gathers and "
+                         "read-modify-writes (the recurrence's access pattern) and exit")
     return ap.parse_args()
 
 
@@ -54,6 +57,29 @@ def peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one k_recur
+# launch per token-head, from an ncu capture of the pages-scale workload at
+# T = 1024 (8192 token-heads; profiles/k_recur_dram_pages_scale_T1024.md),
+# valid for the recurrence source it was taken on.
+RECUR_DRAM_BYTES_PER_TOKEN_HEAD = (270842624 + 90233344) / 8192.0
+RECUR_DRAM_SOURCE_SHA256 = "a351cdd54ab4e2400e450e4ce7dd4d3e5984c88df57dcf0f967ea0e73e96a609"
+
+
+def recur_traffic(token_heads: int):
+    """Per-launch DRAM traffic of k_recur scaled from the capture, or None when
+    the recurrence source changed since the counters were taken."""
+    import hashlib
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                       "sparse_memory_linear_scoring_b200", "csrc", "recur.cu")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if sha != RECUR_DRAM_SOURCE_SHA256:
+        return None
+    return RECUR_DRAM_BYTES_PER_TOKEN_HEAD * token_heads
 
 
 def host_threads() -> int:
@@ -130,13 +156,17 @@ def cpu_baseline(cfg, target_s: float, b0: int = 0):
     nthr = host_threads()
     nheads = min(cfg.BH, nthr)
     sub = cfg.with_(B=1, H=1)
-    # calibrate on one head
-    one = gen_inputs(sub, t_end=16, b0=b0)
-    npi = {k: v.numpy() for k, v in one.items()}
-    d = dict(cfg.dims(), B=1, H=1, T=16)
-    t = time.perf_counter()
-    oracle.forward(npi, d)
-    per_step = (time.perf_counter() - t) / 16
+    # calibrate on one head: the marginal cost of a step (the difference of a
+    # 16- and a 64-step run; the fixed cost of a call is the table's copy)
+    def run_one(steps):
+        one = gen_inputs(sub, t_end=steps, b0=b0)
+        npi = {k: v.numpy() for k, v in one.items()}
+        d = dict(cfg.dims(), B=1, H=1, T=steps)
+        t = time.perf_counter()
+        oracle.forward(npi, d)
+        return time.perf_counter() - t
+    t16, t64 = run_one(16), run_one(64)
+    per_step = max((t64 - t16) / 48, t64 / 64 / 10)
     waves = (nheads + nthr - 1) // nthr
     T_s = int(max(16, min(cfg.T, target_s / max(per_step * waves, 1e-9))))
     heads = [(hh // cfg.H, hh % cfg.H) for hh in range(nheads)]
@@ -295,7 +325,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
                 "achieved": (score_flops / (per[dom] / 1e3) / 1e12) if dom == "score" else None,
                 "peak": fp32_peak, "unit": "TFLOP/s"}
     roof["frac"] = (roof["achieved"] / roof["peak"]) if roof["achieved"] else None
-    roof["traffic"] = None
+    roof["traffic"] = recur_traffic(th) if roof["kernel"] == "k_recur" else None
     roof["peak_source"] = src
     rec_gbs = slot_bytes / (per["recur"] / 1e3) / 1e9
     out = {
@@ -359,8 +389,40 @@ def run_reference(args, cfg):
                     "d2h_bytes_per_step": 0}}
 
 
+def probe_rows():
+    """Random whole-row gathers / read-modify-writes on a 2 GiB table (the size of
+    the pages-scale slot tables), timed with CUDA events after a warm-up launch."""
+    import torch
+    import sparse_memory_linear_scoring_b200 as sdm
+    nrows = 8 << 20
+    table = torch.zeros(nrows, 64, dtype=torch.float32, device="cuda")
+    res = []
+    for ctas in (296, 444, 592):
+        for rmw in (False, True):
+            for u in (4, 8):
+                iters = 64
+                sdm.probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=4)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                sdm.probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=iters)
+                e1.record()
+                e1.synchronize()
+                ms = e0.elapsed_time(e1)
+                nbytes = ctas * 32 * u * iters * 256 * (2 if rmw else 1)
+                res.append({"pattern": "rmw" if rmw else "gather", "rows_in_flight": u,
+                            "ctas": ctas, "ms": ms, "GB/s": nbytes / ms / 1e6})
+    pk, src = peaks()
+    best = {pat: max(r["GB/s"] for r in res if r["pattern"] == pat) for pat in ("gather", "rmw")}
+    return {"probe": "random 256-byte rows of a 2 GiB float32 table", "results": res,
+            "best_GB/s": best, "copy_peak_GB/s": pk["hbm_gbs"], "peak_source": src}
+
+
 def main():
     args = parse()
+    if args.probe_rows:
+        print(json.dumps(probe_rows()), flush=True)
+        return 0
     from synth import config
     cfg = config(args.config)
     if args.T > 0:

@@ -191,3 +191,17 @@ def test_recur_flags_bad_lists():
               n_sub=cfg.n_sub, topk=cfg.k)
     st, info = sdm.device_status()
     assert st & 8 and info == 5
+
+
+def test_probe_random_rows():
+    """The random-row bandwidth probe: gathers leave the table unchanged,
+    read-modify-writes add to it; bad arguments are rejected."""
+    table = torch.zeros(4096, 64, dtype=torch.float32, device="cuda")
+    sdm.probe_random_rows(table, rmw=False, rows_in_flight=4, ctas=2, iters=2)
+    torch.cuda.synchronize()
+    assert int((table != 0).sum()) == 0
+    sdm.probe_random_rows(table, rmw=True, rows_in_flight=8, ctas=2, iters=2)
+    torch.cuda.synchronize()
+    assert float(table.sum()) > 0
+    with pytest.raises(sdm.SDMError):
+        sdm.probe_random_rows(table, rmw=True, rows_in_flight=3, ctas=2, iters=2)
