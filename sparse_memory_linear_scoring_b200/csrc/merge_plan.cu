@@ -45,7 +45,7 @@ __host__ __device__ inline int p2(int x) {
 __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~size_t(15); }
 
 // k_merge: staircase tables, then per warp: two sorted half lists (h1, h2),
-// the candidate scores and two select buffers (32-bit), and the selection.
+// the selection, the candidate scores and cells, and two select buffers.
 struct MergeLayout {
   size_t stair, uni, total, per_warp;
   int Sk, Sc, Ss, warps;
@@ -56,12 +56,12 @@ __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   L.Sk = p2(p.k);
   L.Sc = ((p.ncW > p.ncR ? p.ncW : p.ncR) + 31) & ~31;
   L.Ss = p2(p.W > p.R ? p.W : p.R);
-  if (L.Ss < L.Sc) L.Ss = L.Sc;
   L.warps = warps;
   size_t o = 0;
   L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR) * 4);
   L.uni = o;
-  L.per_warp = size_t(2 * L.Sk + L.Ss) * 8 + size_t(3 * L.Sc) * 4;
+  // h1, h2 [Sk], sel [Ss] (64-bit); cand, cell [Sc], select scratch [2 Sc] (32-bit)
+  L.per_warp = size_t(2 * L.Sk + L.Ss) * 8 + size_t(4 * L.Sc) * 4;
   o += L.per_warp * warps;
   L.total = al16(o);
   return L;
@@ -241,10 +241,10 @@ __device__ uint32_t warp_select32(const uint32_t* cand, int n, int r, uint32_t* 
 // survivor list) -> the n_sel selected slots and their softmax weights.
 // Selection order is unspecified unless `sorted` is set (then rank order).
 __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
-                          int n_sel, const uint32_t* stair, int nc, const uint32_t* front, int nf,
-                          uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* alt,
-                          uint64_t* sel, bool sorted, float* w_out, uint32_t* slot_out,
-                          DevStatus* st, int info) {
+                          int n_sel, const uint32_t* stair, int n_stair, const uint32_t* front,
+                          int nf, uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* cell,
+                          uint32_t* alt, uint64_t* sel, bool sorted, float* w_out,
+                          uint32_t* slot_out, DevStatus* st, int info) {
   const int lane = threadIdx.x & 31;
   if (c1 < p.k || c1 > p.C || c2 < p.k || c2 > p.C) {
     if (lane == 0) dev_flag(st, SDM_DEV_CAPACITY, info);
@@ -259,10 +259,34 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
   }
   __syncwarp();
   const uint32_t n = uint32_t(p.n);
-  // staircase candidate scores (ordered 32-bit images of the float32 sums)
-  for (int i = lane; i < nc; i += 32) {
-    const uint32_t ab = stair[i];
-    cand[i] = f2ord(key_val(h1[ab & 0xffff]) + key_val(h2[ab >> 16]));
+  // A lower bound on the n_sel-th best candidate: all d * e >= n_sel cells of
+  // the d x e corner score at least s1[d-1] + s2[e-1] (sums fall along rows and
+  // columns, and float32 addition is monotone).
+  uint32_t lb = 0;
+  for (int d = lane + 1; d <= p.k; d += 32) {
+    const int e = (n_sel + d - 1) / d;
+    if (e <= p.k) lb = max(lb, f2ord(key_val(h1[d - 1]) + key_val(h2[e - 1])));
+  }
+  lb = __reduce_max_sync(0xffffffffu, lb);
+  // candidates: the staircase cells scoring >= lb (ordered 32-bit images of the
+  // float32 sums) and their cells; they include every staircase cell that
+  // scores >= the n_sel-th best
+  int nc = 0;
+  for (int i0 = 0; i0 < n_stair; i0 += 32) {
+    const int i = i0 + lane;
+    uint32_t x = 0, ab = 0;
+    if (i < n_stair) {
+      ab = stair[i];
+      x = f2ord(key_val(h1[ab & 0xffff]) + key_val(h2[ab >> 16]));
+    }
+    const bool keep = i < n_stair && x >= lb;
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = nc + __popc(m & lanemask_lt());
+      cand[pos] = x;
+      cell[pos] = ab;
+    }
+    nc += __popc(m);
   }
   __syncwarp();
   const uint32_t vstar = warp_select32(cand, nc, n_sel, alt, alt + (nc + 31) / 32 * 32);
@@ -320,7 +344,7 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
         const bool take = (i < nc) && cand[i] > vstar;
         const unsigned m = __ballot_sync(0xffffffffu, take);
         if (take) {
-          const uint32_t ab = stair[i];
+          const uint32_t ab = cell[i];
           const uint64_t a = h1[ab & 0xffff], b = h2[ab >> 16];
           sel[base + __popc(m & lanemask_lt())] =
               (uint64_t(cand[i]) << 32) | uint64_t(~(key_idx(a) * n + key_idx(b)));
@@ -337,7 +361,7 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
       const bool take = (i < nc) && cand[i] >= vstar;
       const unsigned m = __ballot_sync(0xffffffffu, take);
       if (take) {
-        const uint32_t ab = stair[i];
+        const uint32_t ab = cell[i];
         const uint64_t a = h1[ab & 0xffff], b = h2[ab >> 16];
         sel[base + __popc(m & lanemask_lt())] =
             (uint64_t(cand[i]) << 32) | uint64_t(~(key_idx(a) * n + key_idx(b)));
@@ -354,13 +378,18 @@ __device__ void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* 
   }
   // softmax over the selected float32 scores; the best candidate is (0, 0)
   const float m = key_val(h1[0]) + key_val(h2[0]);
+  float* ex = reinterpret_cast<float*>(cand);  // free again (n_sel <= Sc)
   float zs = 0.f;
-  for (int i = lane; i < n_sel; i += 32) zs += expf(key_val(sel[i]) - m);
+  for (int i = lane; i < n_sel; i += 32) {
+    const float e = expf(key_val(sel[i]) - m);
+    ex[i] = e;
+    zs += e;
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
   const float inv = 1.f / zs;
   for (int i = lane; i < n_sel; i += 32) {
-    w_out[i] = expf(key_val(sel[i]) - m) * inv;
+    w_out[i] = ex[i] * inv;
     slot_out[i] = key_idx(sel[i]);
   }
   __syncwarp();
@@ -419,7 +448,8 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   uint64_t* h2 = h1 + L.Sk;
   uint64_t* sel = h2 + L.Sk;
   uint32_t* cand = reinterpret_cast<uint32_t*>(sel + L.Ss);
-  uint32_t* alt = cand + L.Sc;
+  uint32_t* cell = cand + L.Sc;
+  uint32_t* alt = cell + L.Sc;
   for (int pi = warp; pi < 2 * np; pi += kMergeWarps) {
     const int tc = s0 + (pi >> 1), side = pi & 1;
     const size_t hr = (size_t(bh) * p.Tc + tc) * 4 + side * 2;
@@ -429,7 +459,7 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     uint32_t* s_out = reinterpret_cast<uint32_t*>(side ? io.out_ir : io.out_iw) + row * n_sel;
     merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
               io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
-              side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, alt, sel,
+              side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, cell, alt, sel,
               io.sorted != 0, w_out, s_out, st, int(hr));
   }
 }
