@@ -205,3 +205,61 @@ def test_probe_random_rows():
     assert float(table.sum()) > 0
     with pytest.raises(sdm.SDMError):
         sdm.probe_random_rows(table, rmw=True, rows_in_flight=3, ctas=2, iters=2)
+
+
+def _repeat_inputs(cfg, period, share_qk):
+    """Keys (and queries, with share_qk) that repeat with the given period, so
+    the same slots come back every few steps: long runs of one slot inside a
+    plan block, runs crossing chunk and block edges."""
+    inp = gen_inputs(cfg)
+    T = cfg.T
+    idx = torch.arange(T) % period
+    inp["k"] = inp["k"][:, :, idx].contiguous()
+    if share_qk:
+        inp["q"] = inp["k"].clone()
+    return inp
+
+
+@pytest.mark.parametrize("period,share", [(1, True), (3, False), (5, True), (64, True)])
+def test_repeated_slots(period, share):
+    cfg = config(1).with_(B=1, H=2, T=300, n_sub=64, k=16, W=32, R=32, m0_sd=0.5,
+                          in_dtype="f32")
+    inp = _repeat_inputs(cfg, period, share)
+    ref = oracle_full(inp, cfg, lists=True)
+    _check_forward(cfg, inp, ref)
+
+
+def test_all_zero_keys_and_queries():
+    """Every score is 0: every step selects the lowest slots (ties go to the
+    lower index), so each plan block holds the same few slots P times over."""
+    cfg = config(1).with_(B=1, H=2, T=200, n_sub=64, k=16, W=24, R=16, m0_sd=0.5)
+    inp = gen_inputs(cfg)
+    inp["q"] = torch.zeros_like(inp["q"])
+    inp["k"] = torch.zeros_like(inp["k"])
+    ref = oracle_full(inp, cfg, lists=True)
+    assert (ref["idx_w"] == np.sort(ref["idx_w"][0, 0, 0])).all()
+    _check_forward(cfg, inp, ref)
+
+
+@pytest.mark.parametrize("split", [1, 77, 128, 299])
+def test_streaming_split(split):
+    """Two calls over [0, s) and [s, T) with M carried equal one call over
+    [0, T): M bit for bit (the same updates in the same order per slot), o
+    within float32 reduction-order rounding."""
+    cfg = config(1).with_(B=1, H=2, T=300, n_sub=256, k=32, W=64, R=64, m0_sd=0.5)
+    inp = gen_inputs(cfg)
+    d = to_device(inp, cfg)
+    o1, M1 = gpu_forward(d, cfg)
+    M2 = d["M"].clone()
+    parts = []
+    for lo, hi in ((0, split), (split, cfg.T)):
+        sl = {n: (d[n][:, :, lo:hi].contiguous() if n in ("q", "k", "v", "alpha", "beta")
+                  else d[n]) for n in d}
+        parts.append(sdm.forward(sl["q"], sl["k"], sl["v"], sl["alpha"], sl["beta"], sl["C1"],
+                                 sl["C2"], M2, topk=cfg.k, W=cfg.W, R=cfg.R))
+    torch.cuda.synchronize()
+    _status_clean()
+    o2 = torch.cat(parts, dim=2)
+    assert torch.equal(M1, M2)
+    err = (o1 - o2).abs().max().item() / max(o1.abs().max().item(), 1e-30)
+    assert err <= 1e-6, err
