@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time single-step calls (T = 1, M carried), eagerly and as one CUDA "
+                         "graph of --steps steps, on the workload's heads, and exit")
     ap.add_argument("--probe-rows", action="store_true",
                     help="measure the HBM ceiling of random 256-byte row gathers and "
                          "read-modify-writes (the recurrence's access pattern) and exit")
@@ -418,8 +421,70 @@ def probe_rows():
             "best_GB/s": best, "copy_peak_GB/s": pk["hbm_gbs"], "peak_source": src}
 
 
+def decode(cfg, steps):
+    """Streaming use: one sdm_forward call per step (T = 1) with M carried, on
+    the workload's B x H heads; eager launches and one CUDA graph of all steps."""
+    import torch
+    import sparse_memory_linear_scoring_b200 as sdm
+    from synth import gen_inputs
+    inp = gen_inputs(cfg.with_(T=steps), device="cuda")
+    dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
+    per = {}
+    for n in ("q", "k", "v", "alpha", "beta"):
+        x = inp[n].to(dt) if n in ("q", "k", "v") else inp[n]
+        x = x.unsqueeze(-1) if x.dim() == 3 else x          # [B, H, T, d]
+        per[n] = x.permute(2, 0, 1, 3).contiguous().unsqueeze(3)  # [T, B, H, 1, d]
+    C1, C2 = inp["C1"].to(dt).contiguous(), inp["C2"].to(dt).contiguous()
+    M = inp["M0"].contiguous()
+    dims = sdm.make_dims(**cfg.with_(T=1).dims())
+    ws = torch.empty(sdm.workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    o = torch.empty(steps, cfg.B, cfg.H, 1, cfg.d_v, dtype=torch.float32, device="cuda")
+
+    def one(t):
+        a = per["alpha"][t].squeeze(-1)
+        b = per["beta"][t].squeeze(-1)
+        sdm.forward(per["q"][t], per["k"][t], per["v"][t], a, b, C1, C2, M, topk=cfg.k,
+                    W=cfg.W, R=cfg.R, o=o[t], workspace=ws)
+
+    for t in range(min(steps, 8)):
+        one(t)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(steps):
+        one(t)
+    e1.record()
+    e1.synchronize()
+    eager_us = e0.elapsed_time(e1) * 1e3 / steps
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for t in range(steps):
+                one(t)
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    g.replay()
+    e1.record()
+    e1.synchronize()
+    graph_us = e0.elapsed_time(e1) * 1e3 / steps
+    st, info = sdm.device_status(ws)
+    del g
+    return {"decode": "sdm_forward per step (T = 1), M carried", "workload": workload_desc(cfg),
+            "steps": steps, "heads": cfg.BH, "eager_us_per_step": eager_us,
+            "graph_us_per_step": graph_us,
+            "graph_token_heads_per_s": cfg.BH / (graph_us * 1e-6), "device_status": st}
+
+
 def main():
     args = parse()
+    if args.decode:
+        from synth import config as _config
+        print(json.dumps(decode(_config(args.config), max(16, args.steps))), flush=True)
+        return 0
     if args.probe_rows:
         print(json.dumps(probe_rows()), flush=True)
         return 0

@@ -366,6 +366,9 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       const float sd = sqrtf(fmaxf(S2 / m - mu * mu, 0.f));
       if (!keep_all) tau = mu + a.z * sd;
       redo = !keep_all && !(sd > 0.f);
+      // rows past the end of the chunk keep nothing, so that a warp whose rows
+      // are all past it skips the appends (single steps, ragged last tiles)
+      if (!valid) tau = INFINITY;
     }
     // filter: append the kept scores of this thread's columns to the row's list
     float kmin = INFINITY, kmax = -INFINITY;

@@ -195,7 +195,9 @@ static cudaError_t score_chunk(const Plan& p, const Carve& c, const void* q, con
                                const void* C1, const void* C2, int t0, int tlen, cudaStream_t s) {
   cudaError_t e;
   if (p.tc) {
-    if ((e = launch_reset_redo(c.st, s)) != cudaSuccess) return e;
+    // the redo list of the tensor-core filter starts empty in every chunk (the
+    // first chunk's was emptied with the status word)
+    if (t0 > 0 && (e = launch_reset_redo(c.st, s)) != cudaSuccess) return e;
     if ((e = launch_score_tc(p, q, k, C1, C2, t0, tlen, c.cnt, c.surv, c.redo, c.st, s)) !=
         cudaSuccess)
       return e;
@@ -290,8 +292,8 @@ extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
   const int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
   const int64_t per_chunk = (p.tc ? 3 : 1) + 3;
-  const int64_t vals[8] = {p.tc, p.C, p.P, p.S, p.Tc, p.nchunks, 1 + per_chunk * p.nchunks,
-                           p.NB};
+  const int64_t launches = 1 + per_chunk * p.nchunks - (p.tc && p.nchunks > 0 ? 1 : 0);
+  const int64_t vals[8] = {p.tc, p.C, p.P, p.S, p.Tc, p.nchunks, launches, p.NB};
   for (int i = 0; i < n && i < 8; ++i) out[i] = vals[i];
   return SDM_OK;
 }
