@@ -200,13 +200,24 @@ def run_sdm(args, cfg, rank, world, local_rank):
     plan = sdm.query_plan(dims)
     # weak scaling: rank r owns batch rows [r*B, (r+1)*B) of a world*B batch
     b0, _ = shard_batch(cfg.B * world, world, rank)
-    inp = gen_inputs(cfg, b0=b0)
     dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
-    d = {n: inp[n].to(dev, dt).contiguous() for n in ("q", "k", "v", "C1", "C2")}
-    for n in ("alpha", "beta"):
-        d[n] = inp[n].to(dev).contiguous()
-    M = inp["M0"].to(dev).contiguous()
-    del inp
+    # inputs made on the device by the seeded generator, one batch row at a
+    # time (the high-batch table is 64 GiB)
+    d = {}
+    M = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d_v, dtype=torch.float32, device=dev)
+    for b in range(cfg.B):
+        part = gen_inputs(cfg.with_(B=1), device=str(dev), b0=b0 + b)
+        for n in ("q", "k", "v", "alpha", "beta"):
+            if n not in d:
+                shape = (cfg.B,) + tuple(part[n].shape[1:])
+                d[n] = torch.empty(shape, dtype=dt if n in ("q", "k", "v") else torch.float32,
+                                   device=dev)
+            d[n][b] = part[n][0]
+        M[b] = part["M0"][0]
+        if b == 0:
+            d["C1"] = part["C1"].to(dt).contiguous()
+            d["C2"] = part["C2"].to(dt).contiguous()
+        del part
     o = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     nph = 5 * plan["chunks"]

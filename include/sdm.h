@@ -98,7 +98,8 @@ enum {
  * `dims` (0 if dims are invalid).  Depends on dims only.  The workspace
  * holds per-call scratch (per-half survivor lists, the write/read plans of
  * the recurrence, a status word); its contents need not be initialised and
- * are overwritten by each call.
+ * are overwritten by each call.  Long sequences run as several time chunks,
+ * so that it stays near 4 GiB at most.
  */
 SDM_API size_t sdm_workspace_bytes(const sdm_dims* dims);
 

@@ -187,7 +187,8 @@ struct RecurSmem {
 template <typename Tv, int LPR, int F>
 __global__ void __launch_bounds__(kRecurThreads, kRecurWarps / 148 / (kRecurThreads / 32))
 k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restrict__ o,
-        const int4* __restrict__ rec, const int* __restrict__ roff, int t0, int tlen) {
+        const int4* __restrict__ rec, const int* __restrict__ roff, int t0, int tlen, int bh0,
+        int nbh) {
   using SM = RecurSmem<Tv, LPR, F>;
   constexpr int dv = LPR * F;
   constexpr int U = SM::U;
@@ -202,8 +203,8 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
   Tv* vrow = reinterpret_cast<Tv*>(mine + SM::ring + SM::mrow) + sl * F;  // [U][dv], own part
   const unsigned gmask =
       LPR == 32 ? 0xffffffffu : (((1u << LPR) - 1u) << ((threadIdx.x & 31) / LPR * LPR));
-  const int bh = stream / p.S, s = stream - bh * p.S;
-  if (bh >= p.BH) return;  // whole lane groups leave together
+  const int bh = bh0 + stream / p.S, s = stream % p.S;
+  if (bh >= bh0 + nbh) return;  // whole lane groups leave together
   const int nb = (tlen + p.P - 1) / p.P;
   const int g0 = s * p.mb, g1 = g0 + p.mb;
   float* Mh = M + size_t(bh) * size_t(p.N) * dv + sl * F;
@@ -391,11 +392,17 @@ static cudaError_t launch_recur_t(const Plan& p, const void* v, float* M, float*
   cudaError_t e = cudaFuncSetAttribute(k_recur<Tv, LPR, F>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  const long long threads = (long long)p.BH * p.S * LPR;
-  const int grid = int((threads + kRecurThreads - 1) / kRecurThreads);
-  k_recur<Tv, LPR, F><<<grid, kRecurThreads, smem, s>>>(p, (const Tv*)v, M, o, rec, roff, t0,
-                                                        tlen);
-  return cudaGetLastError();
+  // heads in groups of p.HG per launch, so that the rows in use at a time
+  // span a bounded range of the table (address translation reach)
+  for (int bh0 = 0; bh0 < p.BH; bh0 += p.HG) {
+    const int nbh = min(p.HG, p.BH - bh0);
+    const long long threads = (long long)nbh * p.S * LPR;
+    const int grid = int((threads + kRecurThreads - 1) / kRecurThreads);
+    k_recur<Tv, LPR, F><<<grid, kRecurThreads, smem, s>>>(p, (const Tv*)v, M, o, rec, roff, t0,
+                                                          tlen, bh0, nbh);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // Floats per lane F for a row width: kRecurMaxF, kept within [d_v / 32, d_v / 4]

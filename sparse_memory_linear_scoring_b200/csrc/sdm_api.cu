@@ -82,8 +82,14 @@ int make_plan(const sdm_dims* d, Plan* p) {
   // recurrence streams per head: fill the target warp count (a warp holds
   // 32 / LPR streams), keeping at least kStreamMin records per stream and block
   {
+    // heads per recurrence launch: their tables span at most kRecurGroupBytes
+    const size_t table = size_t(p->N) * p->dv * 4;
+    long long HG = (long long)(kRecurGroupBytes / (table > 0 ? table : 1));
+    if (HG < 1) HG = 1;
+    if (HG > p->BH) HG = p->BH;
+    p->HG = int(HG);
     const long long per_warp = 32 / recur_lanes_per_row(p->dv);
-    long long S = (kRecurWarps * per_warp + p->BH - 1) / p->BH;
+    long long S = (kRecurWarps * per_warp + HG - 1) / HG;
     const long long smax = p->E / kStreamMin > 1 ? p->E / kStreamMin : 1;
     if (S > smax) S = smax;
     if (S < 1) S = 1;
@@ -291,7 +297,7 @@ extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
   Plan p;
   const int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
-  const int64_t per_chunk = (p.tc ? 3 : 1) + 3;
+  const int64_t per_chunk = (p.tc ? 3 : 1) + 2 + (p.BH + p.HG - 1) / p.HG;
   const int64_t launches = 1 + per_chunk * p.nchunks - (p.tc && p.nchunks > 0 ? 1 : 0);
   const int64_t vals[8] = {p.tc, p.C, p.P, p.S, p.Tc, p.nchunks, launches, p.NB};
   for (int i = 0; i < n && i < 8; ++i) out[i] = vals[i];

@@ -36,7 +36,11 @@ constexpr int kEntryBits = 13;          // entry index within a block: < 2^13
 static_assert(kMaxBlockEntries <= (1 << kEntryBits), "entry index must fit its key field");
 constexpr int kBucketTarget = 16;       // mean plan records per bucket aimed for
 constexpr int kStreamMin = 4;           // mean records per stream and block, at least
-constexpr size_t kChunkBudget = size_t(1) << 30;  // workspace bytes per time chunk
+constexpr size_t kChunkBudget = size_t(4) << 30;  // workspace bytes per time chunk
+#ifndef SDM_RECUR_GROUP_BYTES
+#define SDM_RECUR_GROUP_BYTES (size_t(8) << 30)  // slot-table bytes per recurrence launch
+#endif
+constexpr size_t kRecurGroupBytes = SDM_RECUR_GROUP_BYTES;
 constexpr int kPlanThreads = 256;
 constexpr int kMergeWarps = 8;          // merge kernel: warps per CTA
 constexpr int kMergeSteps = 16;         // merge kernel: steps per CTA
@@ -56,6 +60,7 @@ struct Plan {
   int S;       // recurrence streams per head (one warp, or a lane group for d_v < 32)
   int NB;      // slot buckets per head = S * mb; stream s owns buckets [s*mb, (s+1)*mb)
   int mb;
+  int HG;      // heads per recurrence launch
   int ncW, nfW, ncR, nfR;  // staircase / frontier sizes of the merge
   size_t merge_smem, plan_smem, recur_smem, score_smem;
   // workspace byte offsets
