@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-probe", action="store_true",
+                    help="skip the random-row probe of the recurrence's access pattern")
     ap.add_argument("--decode", action="store_true",
                     help="time single-step calls (T = 1, M carried), eagerly and as one CUDA "
                          "graph of --steps steps, on the workload's heads, and exit")
@@ -66,8 +68,8 @@ def peaks():
 # launch per token-head, from an ncu capture of the pages-scale workload at
 # T = 1024 (8192 token-heads; profiles/k_recur_dram_pages_scale_T1024.md),
 # valid for the recurrence source it was taken on.
-RECUR_DRAM_BYTES_PER_TOKEN_HEAD = (270842624 + 90233344) / 8192.0
-RECUR_DRAM_SOURCE_SHA256 = "a351cdd54ab4e2400e450e4ce7dd4d3e5984c88df57dcf0f967ea0e73e96a609"
+RECUR_DRAM_BYTES_PER_TOKEN_HEAD = (270892032 + 89945600) / 8192.0
+RECUR_DRAM_SOURCE_SHA256 = "ce6f96528744c2ecea01b7e144f1718abd36b675eaf6233e5709df5d3240523c"
 
 
 def recur_traffic(token_heads: int):
@@ -338,6 +340,11 @@ def run_sdm(args, cfg, rank, world, local_rank):
                "pipelined": "copies of steps i+1 (in) and i-1 (out) overlap step i",
                "l2": "not flushed: the 2 GiB state is larger than L2"}
 
+    # the random-row ceiling of the recurrence's access pattern, this run
+    pat = None
+    if not args.no_probe:
+        del flush
+        pat = pattern_ceiling(cfg.W, cfg.R)
     if rank != 0:
         return None
     pk, src = peaks()
@@ -380,7 +387,10 @@ def run_sdm(args, cfg, rank, world, local_rank):
         "slot_traffic": {"bytes_per_step": slot_bytes, "recur_gbs": rec_gbs,
                          "recur_frac_of_8TBs": rec_gbs / 8000.0,
                          "recur_frac_of_measured": rec_gbs / pk["hbm_gbs"],
-                         "whole_step_gbs": slot_bytes / (t_max / K / 1e3) / 1e9},
+                         "whole_step_gbs": slot_bytes / (t_max / K / 1e3) / 1e9,
+                         "pattern": pat,
+                         "recur_frac_of_pattern_ceiling":
+                             rec_gbs / pat["ceiling_gbs"] if pat else None},
         "phases_ms": per, "phase_share": shares, "plan": plan,
         "gpu_launches": int(plan["launches_per_call"] * K),
         "clocks": clk, "e2e": e2e,
@@ -430,7 +440,7 @@ def run_reference(args, cfg):
                     "d2h_bytes_per_step": 0}}
 
 
-def probe_rows():
+def probe_rows(configs=None):
     """Random whole-row gathers / read-modify-writes on a 2 GiB table (the size of
     the pages-scale slot tables), timed with CUDA events after a warm-up launch."""
     import torch
@@ -438,9 +448,12 @@ def probe_rows():
     nrows = 8 << 20
     table = torch.zeros(nrows, 64, dtype=torch.float32, device="cuda")
     res = []
-    for ctas in (296, 444, 592):
-        for rmw in (False, True):
-            for u in (4, 8):
+    if configs is None:
+        configs = [(ctas, rmw, u) for ctas in (296, 444, 592) for rmw in (False, True)
+                   for u in (4, 8)]
+    for ctas, rmw, u in configs:
+        if True:
+            if True:
                 iters = 64
                 sdm.probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=4)
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -453,10 +466,22 @@ def probe_rows():
                 nbytes = ctas * 32 * u * iters * 256 * (2 if rmw else 1)
                 res.append({"pattern": "rmw" if rmw else "gather", "rows_in_flight": u,
                             "ctas": ctas, "ms": ms, "GB/s": nbytes / ms / 1e6})
+    del table
     pk, src = peaks()
     best = {pat: max(r["GB/s"] for r in res if r["pattern"] == pat) for pat in ("gather", "rmw")}
     return {"probe": "random 256-byte rows of a 2 GiB float32 table", "results": res,
             "best_GB/s": best, "copy_peak_GB/s": pk["hbm_gbs"], "peak_source": src}
+
+
+def pattern_ceiling(W, R):
+    """The HBM ceiling of the recurrence's own access pattern: 2W of every
+    (2W + R) rows are read-modify-writes, R are gathers (best of a few launch
+    shapes of the random-row probe, measured in the same run)."""
+    pr = probe_rows([(592, False, 8), (296, False, 8), (592, True, 4), (296, True, 8)])
+    g, m = pr["best_GB/s"]["gather"], pr["best_GB/s"]["rmw"]
+    f = 2.0 * W / (2.0 * W + R)
+    return {"gather_gbs": g, "rmw_gbs": m, "rmw_fraction": f,
+            "ceiling_gbs": 1.0 / (f / m + (1.0 - f) / g)}
 
 
 def decode(cfg, steps):
