@@ -41,9 +41,15 @@ constexpr size_t kChunkBudget = size_t(4) << 30;  // workspace bytes per time ch
 #define SDM_RECUR_GROUP_BYTES (size_t(8) << 30)  // slot-table bytes per recurrence launch
 #endif
 constexpr size_t kRecurGroupBytes = SDM_RECUR_GROUP_BYTES;
-constexpr int kPlanThreads = 256;
-constexpr int kMergeWarps = 8;          // merge kernel: warps per CTA
-constexpr int kMergeSteps = 16;         // merge kernel: steps per CTA
+#ifndef SDM_PLAN_THREADS
+#define SDM_PLAN_THREADS 512
+#endif
+#ifndef SDM_MERGE_WARPS
+#define SDM_MERGE_WARPS 8
+#endif
+constexpr int kPlanThreads = SDM_PLAN_THREADS;
+constexpr int kMergeWarps = SDM_MERGE_WARPS;  // merge kernel: warps per CTA
+constexpr int kMergeSteps = 2 * SDM_MERGE_WARPS;  // merge kernel: steps per CTA
 
 // Everything the kernels need to know about one call.
 struct Plan {
