@@ -24,7 +24,7 @@
  *          every other slot is left unchanged;
  *  item 4  the output is the weighted sum of the R read slots.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent, each stated here:
  *  - half scores are dot products taken in float64 from the exact input
  *    values, then rounded to float32 ("fp32 scores");
  *  - ordering is (score descending, index ascending): the lower index wins a
