@@ -7,10 +7,16 @@ bf16 inputs, float32 state.  One step = one full forward pass (scoring,
 selection, gated delta recurrence, reads) over the batch.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdm|reference]
+                  [--config 0..4] [--T steps] [--decode] [--probe-rows]
 
 Prints one JSON line (rank 0).  Under torchrun each rank runs its own shard of
 the batch (weak scaling, no collective on the data path); time is the max over
 ranks of the summed per-step CUDA-event times, with L2 flushed between steps.
+The line also carries: the roofline of the dominant kernel; the random-row
+ceiling of the recurrence's access pattern, measured in the same run; an
+end-to-end rate through the public API with pinned host inputs and outputs
+copied every step (pipelined with the compute, as a serving loop would); and
+the oracle timed on the host cores.  --impl reference times the oracle alone.
 """
 from __future__ import annotations
 
