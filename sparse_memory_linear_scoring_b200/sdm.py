@@ -93,12 +93,13 @@ def _workspace(dims: Dims, device: torch.device, workspace: Optional[torch.Tenso
             raise SDMError(4, "workspace too small or on another device")
         return workspace
     key = (device.index if device.index is not None else torch.cuda.current_device(), need)
-    ws = _ws_cache.get(key)
-    if ws is None:
-        for k_old in [k for k in _ws_cache if k[0] == key[0]]:
-            del _ws_cache[k_old]
-        ws = torch.empty(need, dtype=torch.uint8, device=device)
-        _ws_cache[key] = ws
+    with _lock:
+        ws = _ws_cache.get(key)
+        if ws is None:
+            for k_old in [k for k in _ws_cache if k[0] == key[0]]:
+                del _ws_cache[k_old]
+            ws = torch.empty(need, dtype=torch.uint8, device=device)
+            _ws_cache[key] = ws
     return ws
 
 
