@@ -82,7 +82,7 @@ enum {
   SDM_ERR_UNSUPPORTED = 5, /* valid sizes this build has no kernel for */
   SDM_ERR_CUDA = 6,        /* a CUDA call failed while enqueueing */
   SDM_ERR_DEVICE = 7,      /* a kernel's own check fired (see sdm_get_device_status) */
-  SDM_ERR_SCRATCH_LIMIT = 8 /* sdm_forward_noalloc: problem needs more than its 64 MiB scratch */
+  SDM_ERR_SCRATCH_LIMIT = 8 /* sdm_forward_noalloc: problem does not fit its 64 MiB scratch */
 };
 
 /* Device status bits recorded by the kernels (sdm_get_device_status). */
@@ -161,17 +161,20 @@ SDM_API int sdm_forward_timed(const void* q, const void* k, const void* v, const
  * imply.  The pages have no counterpart; this is an interface convenience.
  *
  * Its scratch is one file-scope device array of 64 MiB that every GPU loading
- * this library holds until the process exits.  Problems whose
- * sdm_workspace_bytes(dims) exceeds 64 MiB are rejected with
+ * this library holds until the process exits.  The call runs in time chunks
+ * short enough for its scratch to fit there (the results do not depend on the
+ * chunk length); a problem that does not fit even with the shortest chunk (one
+ * plan block of steps, see sdm_query_plan) is rejected with
  * SDM_ERR_SCRATCH_LIMIT before anything is enqueued.  Runs on the current
- * device; `stream` must belong to it.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  Every call shares the one
- * array and it keeps the last call's contents (nothing in it needs to start
- * at zero), so calls that overlap on the GPU race: serialise them (one stream,
- * or events).  The kernels' status word is not readable through this entry
- * point.  Allocates nothing (no cudaMalloc, cudaFree or allocating library
- * call).  Results and other return codes as sdm_forward.
+ * device; `stream` must belong to it.  Every call looks up the array's device
+ * address (cudaGetSymbolAddress, which allocates nothing) with that device
+ * current; the first call on a device may also load the library's device
+ * code, so make it before any stream capture.  Every call shares the one array
+ * and it keeps the last call's contents (nothing in it needs to start at
+ * zero), so calls that overlap on the GPU race: serialise them (one stream, or
+ * events).  The kernels' status word is not readable through this entry point.
+ * Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * Results and other return codes as sdm_forward.
  */
 SDM_API int sdm_forward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
                                 const float* beta, const void* C1, const void* C2,

@@ -22,8 +22,9 @@
 // A row whose kept count falls outside [k, capacity] (or whose scores do not
 // spread) is queued for the exact CUDA-core path instead, so the result is
 // exact for any input.  Every mbarrier wait is bounded: on a timeout the CTA
-// records SDM_DEV_TIMEOUT, stops issuing work, drains what it issued (bounded)
-// and frees its TMEM.
+// records SDM_DEV_TIMEOUT, stops issuing work, drains what it issued (bounded),
+// frees its TMEM and queues all of its rows for the exact path, so that the
+// selection stays exact even then.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -417,7 +418,10 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
     const int k = p.k;
     const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
     bool go = ok && valid && !redo && cnt >= k && cnt <= C;
-    if (ok && valid && !go && sub == 0) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+    // every valid row this CTA does not settle -- including all of them after a
+    // timed-out wait -- is re-scored exactly, so no later kernel reads a list
+    // this call never wrote
+    if (valid && !go && sub == 0) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
     float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
     for (int j = 0; j < kQ; ++j) {

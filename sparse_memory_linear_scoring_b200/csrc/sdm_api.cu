@@ -49,7 +49,7 @@ static bool dv_supported(int dv) {
   return dv == 4 || dv == 8 || dv == 16 || dv == 32 || dv == 64 || dv == 128;
 }
 
-int make_plan(const sdm_dims* d, Plan* p) {
+int make_plan(const sdm_dims* d, Plan* p, size_t chunk_budget) {
   if (!d) return SDM_ERR_NULL;
   memset(p, 0, sizeof(*p));
   const long long kk = (long long)d->k * d->k;
@@ -104,7 +104,7 @@ int make_plan(const sdm_dims* d, Plan* p) {
                                            size_t(p->W + p->R) * (16 + 8)) +
                           (size_t(p->BH) * (p->NB + 1) * 4 + size_t(P) - 1) / size_t(P);
   const long long Tround = ((long long)(p->T > 0 ? p->T : 1) + P - 1) / P * P;
-  long long Tc = (long long)(kChunkBudget / per_step) / P * P;
+  long long Tc = (long long)(chunk_budget / per_step) / P * P;
   if (Tc < P) Tc = P;
   if (Tc > Tround) Tc = Tround;
   p->Tc = int(Tc);
@@ -222,12 +222,13 @@ extern "C" size_t sdm_workspace_bytes(const sdm_dims* dims) {
   return p.total;
 }
 
-static int forward_impl(const void* q, const void* k, const void* v, const float* alpha,
-                        const float* beta, const void* C1, const void* C2, float* M_inout,
-                        float* o_out, const sdm_dims* dims, void* workspace, size_t ws_bytes,
-                        void* stream, void* const* events, int n_events) {
+int sdm::forward_with_budget(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const void* C1, const void* C2, float* M_inout,
+                             float* o_out, const sdm_dims* dims, void* workspace,
+                             size_t ws_bytes, void* stream, void* const* events, int n_events,
+                             size_t chunk_budget) {
   Plan p;
-  int rc = make_plan(dims, &p);
+  int rc = make_plan(dims, &p, chunk_budget);
   if (rc != SDM_OK) return rc;
   if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
   rc = check_ptrs({q, k, v, alpha, beta, C1, C2, M_inout, o_out, workspace});
@@ -280,8 +281,8 @@ extern "C" int sdm_forward(const void* q, const void* k, const void* v, const fl
                            const float* beta, const void* C1, const void* C2, float* M_inout,
                            float* o_out, const sdm_dims* dims, void* workspace, size_t ws_bytes,
                            void* stream) {
-  return forward_impl(q, k, v, alpha, beta, C1, C2, M_inout, o_out, dims, workspace, ws_bytes,
-                      stream, nullptr, 0);
+  return forward_with_budget(q, k, v, alpha, beta, C1, C2, M_inout, o_out, dims, workspace,
+                             ws_bytes, stream, nullptr, 0, kChunkBudget);
 }
 
 extern "C" int sdm_forward_timed(const void* q, const void* k, const void* v, const float* alpha,
@@ -289,8 +290,8 @@ extern "C" int sdm_forward_timed(const void* q, const void* k, const void* v, co
                                  float* M_inout, float* o_out, const sdm_dims* dims,
                                  void* workspace, size_t ws_bytes, void* stream,
                                  void* const* events, int n_events) {
-  return forward_impl(q, k, v, alpha, beta, C1, C2, M_inout, o_out, dims, workspace, ws_bytes,
-                      stream, events, n_events);
+  return forward_with_budget(q, k, v, alpha, beta, C1, C2, M_inout, o_out, dims, workspace,
+                             ws_bytes, stream, events, n_events, kChunkBudget);
 }
 
 extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
@@ -393,7 +394,7 @@ extern "C" const char* sdm_status_string(int status) {
     case SDM_ERR_UNSUPPORTED: return "valid sizes without a kernel in this build";
     case SDM_ERR_CUDA: return "a CUDA call failed while enqueueing";
     case SDM_ERR_DEVICE: return "a kernel's own check fired";
-    case SDM_ERR_SCRATCH_LIMIT: return "problem needs more than the 64 MiB static scratch";
+    case SDM_ERR_SCRATCH_LIMIT: return "problem does not fit the 64 MiB static scratch";
     default: return "unknown status";
   }
 }

@@ -81,7 +81,17 @@ struct DevStatus {
   int32_t pad[13];
 };
 
-int make_plan(const sdm_dims* d, Plan* p);  // SDM_OK or an error code
+// SDM_OK or an error code.  chunk_budget bounds the workspace bytes of one
+// time chunk (the default, kChunkBudget, keeps it near 4 GiB); a smaller budget
+// gives shorter chunks and the same results.
+int make_plan(const sdm_dims* d, Plan* p, size_t chunk_budget = kChunkBudget);
+
+// The forward pass of sdm_forward / sdm_forward_timed on a caller workspace
+// laid out by make_plan(d, &p, chunk_budget) (same budget).
+int forward_with_budget(const void* q, const void* k, const void* v, const float* alpha,
+                        const float* beta, const void* C1, const void* C2, float* M_inout,
+                        float* o_out, const sdm_dims* dims, void* workspace, size_t ws_bytes,
+                        void* stream, void* const* events, int n_events, size_t chunk_budget);
 
 // ---- device helpers ---------------------------------------------------------
 __device__ __forceinline__ uint32_t f2ord(float v) {

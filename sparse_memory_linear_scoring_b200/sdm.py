@@ -73,9 +73,17 @@ def _check(rc: int):
         raise SDMError(rc, load_library().sdm_status_string(rc).decode())
 
 
+_IN_DTYPES = {torch.float32: SDM_DTYPE_F32, torch.bfloat16: SDM_DTYPE_BF16}
+
+
 def make_dims(B, H, T, d_qk, d_v, n_sub, k, W, R, in_dtype) -> Dims:
+    """Problem sizes; in_dtype is SDM_DTYPE_F32 / SDM_DTYPE_BF16 or the torch dtype
+    (float32 or bfloat16 only) of q', k', v, C1 and C2."""
     if isinstance(in_dtype, torch.dtype):
-        in_dtype = SDM_DTYPE_BF16 if in_dtype == torch.bfloat16 else SDM_DTYPE_F32
+        if in_dtype not in _IN_DTYPES:
+            raise TypeError("input dtype must be torch.float32 or torch.bfloat16, not %s"
+                            % in_dtype)
+        in_dtype = _IN_DTYPES[in_dtype]
     return Dims(int(B), int(H), int(T), int(d_qk), int(d_v), int(n_sub), int(k), int(W), int(R),
                 int(in_dtype))
 
@@ -89,8 +97,10 @@ def _workspace(dims: Dims, device: torch.device, workspace: Optional[torch.Tenso
     if need == 0:
         _check(load_library().sdm_forward(*([None] * 9), ctypes.byref(dims), None, 0, None))
     if workspace is not None:
-        if workspace.device != device or workspace.numel() * workspace.element_size() < need:
+        if workspace.device != device or _nbytes(workspace) < need:
             raise SDMError(4, "workspace too small or on another device")
+        if not workspace.is_contiguous():
+            raise ValueError("workspace must be contiguous")
         return workspace
     key = (device.index if device.index is not None else torch.cuda.current_device(), need)
     with _lock:
@@ -115,6 +125,60 @@ def _dev(*ts) -> torch.device:
     return dev
 
 
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
+def _expect(t: torch.Tensor, name: str, shape, dtypes) -> None:
+    """Raise before any launch unless `t` has exactly `shape` and one of `dtypes`."""
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if t.dtype not in dtypes:
+        raise TypeError("%s has dtype %s, expected %s" % (name, t.dtype,
+                                                           " or ".join(map(str, dtypes))))
+
+
+def _check_inputs(q, k, v, C1, C2, alpha=None, beta=None):
+    """Shapes and dtypes of the projected inputs; returns (B, H, T, d_qk, n_sub, dtype)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, T, d_qk], got shape %s" % (tuple(q.shape),))
+    B, H, T, d_qk = q.shape
+    if q.dtype not in _IN_DTYPES:
+        raise TypeError("q has dtype %s, expected torch.float32 or torch.bfloat16" % q.dtype)
+    if d_qk % 2:
+        raise ValueError("d_qk = %d must be even" % d_qk)
+    if C1.dim() != 3:
+        raise ValueError("C1 must be [H, n_sub, d_qk/2], got shape %s" % (tuple(C1.shape),))
+    n_sub = C1.shape[1]
+    _expect(k, "k", (B, H, T, d_qk), (q.dtype,))
+    _expect(C1, "C1", (H, n_sub, d_qk // 2), (q.dtype,))
+    _expect(C2, "C2", (H, n_sub, d_qk // 2), (q.dtype,))
+    if v is not None:
+        if v.dim() != 4:
+            raise ValueError("v must be [B, H, T, d_v], got shape %s" % (tuple(v.shape),))
+        _expect(v, "v", (B, H, T, v.shape[-1]), (q.dtype,))
+    for name, t in (("alpha", alpha), ("beta", beta)):
+        if t is not None:
+            _expect(t, name, (B, H, T), (torch.float32,))
+    return B, H, T, d_qk, n_sub, q.dtype
+
+
+def _no_alias(outs, ins) -> None:
+    """Outputs must not overlap each other or any input (raise before any launch)."""
+    def span(t):
+        return t.data_ptr(), t.data_ptr() + _nbytes(t)
+    for i, (no, o) in enumerate(outs):
+        if o.numel() == 0:
+            continue
+        a0, a1 = span(o)
+        for nt, t in list(outs[i + 1:]) + list(ins):
+            if t is None or t.numel() == 0:
+                continue
+            b0, b1 = span(t)
+            if a0 < b1 and b0 < a1:
+                raise ValueError("%s overlaps %s; outputs must not alias other tensors" % (no, nt))
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -123,11 +187,6 @@ def _stream(dev, stream):
     if stream is None:
         stream = torch.cuda.current_stream(dev)
     return ctypes.c_void_p(stream.cuda_stream)
-
-
-def _dims_of(q: torch.Tensor, v: torch.Tensor, C1: torch.Tensor, topk: int, W: int, R: int) -> Dims:
-    B, H, T, d_qk = q.shape
-    return make_dims(B, H, T, d_qk, v.shape[-1], C1.shape[1], topk, W, R, q.dtype)
 
 
 PLAN_FIELDS = ("tensor_core_scoring", "survivor_capacity", "block_steps", "streams_per_head",
@@ -149,22 +208,27 @@ def forward(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
     q, k, v, C1, C2 share one dtype (float32 or bfloat16).  Returns o [B,H,T,d_v] float32.
     events: optional list of torch.cuda.Event recorded at the kernel-phase
     boundaries (see sdm_forward_timed in include/sdm.h)."""
-    dev = _dev(q, k, v, alpha, beta, C1, C2, M)
-    dims = _dims_of(q, v, C1, topk, W, R)
+    B, H, T, d_qk, n_sub, dt = _check_inputs(q, k, v, C1, C2, alpha, beta)
+    d_v = v.shape[-1]
+    _expect(M, "M", (B, H, n_sub * n_sub, d_v), (torch.float32,))
+    if o is not None:
+        _expect(o, "o", (B, H, T, d_v), (torch.float32,))
+    dev = _dev(q, k, v, alpha, beta, C1, C2, M, *([o] if o is not None else []))
+    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, W, R, dt)
     if o is None:
-        o = torch.empty(q.shape[0], q.shape[1], q.shape[2], v.shape[-1], dtype=torch.float32,
-                        device=dev)
-    _dev(o, q)
+        o = torch.empty(B, H, T, d_v, dtype=torch.float32, device=dev)
+    _no_alias([("M", M), ("o", o)], [("q", q), ("k", k), ("v", v), ("alpha", alpha),
+                                     ("beta", beta), ("C1", C1), ("C2", C2)])
     ws = _workspace(dims, dev, workspace)
     lib = load_library()
     if events:
         ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib.sdm_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(C1),
                                      _ptr(C2), _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws),
-                                     ws.numel(), _stream(dev, stream), ev, len(events)))
+                                     _nbytes(ws), _stream(dev, stream), ev, len(events)))
         return o
     _check(lib.sdm_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(C1), _ptr(C2),
-                           _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws), ws.numel(),
+                           _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws), _nbytes(ws),
                            _stream(dev, stream)))
     return o
 
@@ -172,9 +236,9 @@ def forward(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
 def select(q, k, C1, C2, *, topk: int, W: int, R: int, d_v: int = 4,
            workspace: Optional[torch.Tensor] = None, stream=None):
     """Selection lists (item 2): returns idx_w [B,H,T,W] int32, w_w float32, idx_r, w_r."""
+    B, H, T, d_qk, n_sub, dt = _check_inputs(q, k, None, C1, C2)
     dev = _dev(q, k, C1, C2)
-    B, H, T, d_qk = q.shape
-    dims = make_dims(B, H, T, d_qk, d_v, C1.shape[1], topk, W, R, q.dtype)
+    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, W, R, dt)
     idx_w = torch.empty(B, H, T, W, dtype=torch.int32, device=dev)
     w_w = torch.empty(B, H, T, W, dtype=torch.float32, device=dev)
     idx_r = torch.empty(B, H, T, R, dtype=torch.int32, device=dev)
@@ -182,7 +246,7 @@ def select(q, k, C1, C2, *, topk: int, W: int, R: int, d_v: int = 4,
     ws = _workspace(dims, dev, workspace)
     lib = load_library()
     _check(lib.sdm_select(_ptr(q), _ptr(k), _ptr(C1), _ptr(C2), _ptr(idx_w), _ptr(w_w),
-                          _ptr(idx_r), _ptr(w_r), ctypes.byref(dims), _ptr(ws), ws.numel(),
+                          _ptr(idx_r), _ptr(w_r), ctypes.byref(dims), _ptr(ws), _nbytes(ws),
                           _stream(dev, stream)))
     return idx_w, w_w, idx_r, w_r
 
@@ -191,15 +255,33 @@ def recur(v, alpha, beta, idx_w, w_w, idx_r, w_r, M, *, d_qk: int, n_sub: int, t
           o: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
           stream=None) -> torch.Tensor:
     """Recurrence from given lists (items 3-4).  Returns o; M is updated in place."""
-    dev = _dev(v, alpha, beta, idx_w, w_w, idx_r, w_r, M)
+    if v.dim() != 4 or idx_w.dim() != 4 or idx_r.dim() != 4:
+        raise ValueError("v, idx_w and idx_r must be 4-D ([B, H, T, d_v], [B, H, T, W], "
+                         "[B, H, T, R])")
     B, H, T, d_v = v.shape
-    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, idx_w.shape[-1], idx_r.shape[-1], v.dtype)
+    W, R = idx_w.shape[-1], idx_r.shape[-1]
+    if v.dtype not in _IN_DTYPES:
+        raise TypeError("v has dtype %s, expected torch.float32 or torch.bfloat16" % v.dtype)
+    _expect(alpha, "alpha", (B, H, T), (torch.float32,))
+    _expect(beta, "beta", (B, H, T), (torch.float32,))
+    _expect(idx_w, "idx_w", (B, H, T, W), (torch.int32,))
+    _expect(w_w, "w_w", (B, H, T, W), (torch.float32,))
+    _expect(idx_r, "idx_r", (B, H, T, R), (torch.int32,))
+    _expect(w_r, "w_r", (B, H, T, R), (torch.float32,))
+    _expect(M, "M", (B, H, int(n_sub) * int(n_sub), d_v), (torch.float32,))
+    if o is not None:
+        _expect(o, "o", (B, H, T, d_v), (torch.float32,))
+    dev = _dev(v, alpha, beta, idx_w, w_w, idx_r, w_r, M, *([o] if o is not None else []))
+    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, W, R, v.dtype)
     if o is None:
         o = torch.empty(B, H, T, d_v, dtype=torch.float32, device=dev)
+    _no_alias([("M", M), ("o", o)], [("v", v), ("alpha", alpha), ("beta", beta),
+                                     ("idx_w", idx_w), ("w_w", w_w), ("idx_r", idx_r),
+                                     ("w_r", w_r)])
     ws = _workspace(dims, dev, workspace)
     lib = load_library()
     _check(lib.sdm_recur(_ptr(v), _ptr(alpha), _ptr(beta), _ptr(idx_w), _ptr(w_w), _ptr(idx_r),
-                         _ptr(w_r), _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws), ws.numel(),
+                         _ptr(w_r), _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws), _nbytes(ws),
                          _stream(dev, stream)))
     return o
 
@@ -215,7 +297,7 @@ def device_status(workspace: Optional[torch.Tensor] = None, stream=None) -> Tupl
         workspace = cands[-1]
     st = ctypes.c_int32(0)
     info = ctypes.c_int32(0)
-    _check(load_library().sdm_get_device_status(_ptr(workspace), workspace.numel(),
+    _check(load_library().sdm_get_device_status(_ptr(workspace), _nbytes(workspace),
                                                 ctypes.byref(st), ctypes.byref(info),
                                                 _stream(workspace.device, stream)))
     return int(st.value), int(info.value)

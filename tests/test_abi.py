@@ -98,3 +98,73 @@ def test_binding_refuses_cpu_tensors():
         sdm.forward(q, q, torch.zeros(1, 1, 4, 4), torch.zeros(1, 1, 4), torch.zeros(1, 1, 4),
                     torch.zeros(1, 4, 4), torch.zeros(1, 4, 4), torch.zeros(1, 1, 16, 4),
                     topk=2, W=2, R=2)
+
+
+def _cpu_args(**over):
+    """Consistent CPU tensors of a small bf16 problem (B=2, H=3, T=5, d_qk=8,
+    d_v=4, n_sub=4), with named replacements."""
+    import torch
+    B, H, T, dqk, dv, n = 2, 3, 5, 8, 4, 4
+    bf = torch.bfloat16
+    a = dict(q=torch.zeros(B, H, T, dqk, dtype=bf), k=torch.zeros(B, H, T, dqk, dtype=bf),
+             v=torch.zeros(B, H, T, dv, dtype=bf), alpha=torch.zeros(B, H, T),
+             beta=torch.zeros(B, H, T), C1=torch.zeros(H, n, dqk // 2, dtype=bf),
+             C2=torch.zeros(H, n, dqk // 2, dtype=bf), M=torch.zeros(B, H, n * n, dv))
+    a.update(over)
+    return a
+
+
+def _fwd(a, **kw):
+    return sdm.forward(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["C1"], a["C2"], a["M"],
+                       topk=2, W=2, R=2, **kw)
+
+
+@pytest.mark.parametrize("name,bad,exc", [
+    ("q", "float16", TypeError),
+    ("k", (2, 3, 5, 6), ValueError),
+    ("k", "float32", TypeError),
+    ("v", "float32", TypeError),
+    ("v", (2, 3, 4, 4), ValueError),
+    ("alpha", (2, 3, 1), ValueError),
+    ("alpha", "bfloat16", TypeError),
+    ("beta", (3, 2, 5), ValueError),
+    ("C2", (3, 5, 4), ValueError),
+    ("C1", (3, 4, 3), ValueError),
+    ("M", (2, 3, 15, 4), ValueError),
+    ("M", "bfloat16", TypeError),
+])
+def test_binding_rejects_mismatches(name, bad, exc):
+    """Every tensor is checked against the dims before anything is launched (a
+    short M or a float16 input would otherwise reach a kernel)."""
+    import torch
+    a = _cpu_args()
+    if isinstance(bad, str):
+        a[name] = a[name].to(getattr(torch, bad))
+    else:
+        a[name] = torch.zeros(bad, dtype=a[name].dtype)
+    with pytest.raises(exc):
+        _fwd(a)
+
+
+def test_binding_rejects_bad_output_and_lists():
+    import torch
+    a = _cpu_args()
+    with pytest.raises(ValueError):
+        _fwd(a, o=torch.zeros(2, 3, 5, 8))
+    with pytest.raises(TypeError):
+        _fwd(a, o=torch.zeros(2, 3, 5, 4, dtype=torch.float64))
+    with pytest.raises(TypeError):
+        sdm.make_dims(1, 1, 1, 8, 4, 4, 2, 2, 2, torch.float16)
+    B, H, T = 2, 3, 5
+    lists = dict(idx_w=torch.zeros(B, H, T, 2, dtype=torch.int64),
+                 w_w=torch.zeros(B, H, T, 2), idx_r=torch.zeros(B, H, T, 2, dtype=torch.int32),
+                 w_r=torch.zeros(B, H, T, 2))
+    with pytest.raises(TypeError):
+        sdm.recur(a["v"], a["alpha"], a["beta"], lists["idx_w"], lists["w_w"], lists["idx_r"],
+                  lists["w_r"], a["M"], d_qk=8, n_sub=4, topk=2)
+    lists["idx_w"] = lists["idx_w"].to(torch.int32)
+    with pytest.raises(ValueError):
+        sdm.recur(a["v"], a["alpha"], a["beta"], lists["idx_w"], lists["w_w"], lists["idx_r"],
+                  torch.zeros(B, H, T, 3), a["M"], d_qk=8, n_sub=4, topk=2)
+    with pytest.raises(ValueError):
+        sdm.select(a["q"], a["k"][:, :, :4], a["C1"], a["C2"], topk=2, W=2, R=2)

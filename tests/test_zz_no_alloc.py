@@ -3,9 +3,11 @@ memory (its scratch is a fixed 64 MiB device array inside the library).
 
 Called through the C ABI twice in a row, it must give the results of the
 workspace-taking entry point sdm_forward within the parity tolerance (1e-4
-relative per head), and it must refuse a problem whose scratch exceeds the
-array.  This file is collected last so that a failure here comes after every
-other test has run."""
+relative per head), on CUDA-core and tensor-core scoring shapes and on a
+workload whose usual workspace is larger than the array (it then runs in
+shorter time chunks); and it must refuse a problem that does not fit the array
+even in the shortest chunks.  This file is collected last so that a failure
+here comes after every other test has run."""
 import ctypes
 
 import numpy as np
@@ -39,13 +41,19 @@ def _call(fn, d, M, o, dims):
 @pytest.mark.parametrize("cfg", [
     config(0).with_(m0_sd=0.5),
     config(1).with_(B=1, H=2, T=300, n_sub=64, k=16, W=32, R=32, m0_sd=0.5),
-], ids=["tiny-fp32", "small-bf16"])
+    config(1).with_(B=1, H=2, T=300, n_sub=256, k=32, W=64, R=64, m0_sd=0.5),
+    config(1).with_(m0_sd=0.5),
+], ids=["tiny-fp32", "small-bf16-cuda-cores", "small-bf16-tensor-cores", "small-full-chunked"])
 def test_noalloc_matches_forward(cfg):
     fn = _lib()
     inp = gen_inputs(cfg)
     d = to_device(inp, cfg)
     dims = sdm.make_dims(**cfg.dims())
-    assert sdm.workspace_bytes(dims) <= 64 << 20
+    if cfg.n_sub == 256:
+        assert sdm.query_plan(dims)["tensor_core_scoring"] == 1
+    if cfg.B == 4:
+        # its one-chunk workspace (~194 MiB) exceeds the array: shorter chunks
+        assert sdm.workspace_bytes(dims) > 64 << 20
     M_ref = d["M"].clone()
     o_ref = sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], M_ref,
                         topk=cfg.k, W=cfg.W, R=cfg.R)
@@ -61,7 +69,8 @@ def test_noalloc_matches_forward(cfg):
 
 def test_noalloc_rejects_oversize():
     fn = _lib()
-    cfg = config(1)                          # needs ~194 MiB of scratch
+    # 1024 heads: one plan block of steps alone needs ~0.5 GiB of scratch
+    cfg = config(4)
     dims = sdm.make_dims(**cfg.dims())
     assert sdm.workspace_bytes(dims) > 64 << 20
     t = torch.zeros(16, device="cuda")
