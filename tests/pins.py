@@ -15,7 +15,12 @@ build) and raises AssertionError when the oracle disagrees with:
     slot numbering i1*n + i2;
   * invariants: unselected rows stay bit-identical; splitting the time axis
     with the table carried over gives bit-identical results;
-  * W = R = N (k = n): a dense all-slot gated delta update written with numpy.
+  * W = R = N (k = n): a dense all-slot gated delta update written with numpy;
+  * the near-tie flags, from their definition in the workload specification (a
+    float64 gap below 1e-5 relative at the W-th/(W+1)-th (R-th/(R+1)-th)
+    candidate, or at a half's k-th/(k+1)-th row): hand-built score tables whose
+    gaps are known by construction, just below and just above the threshold,
+    for each bit.
 The same functions are run against deliberately broken copies of the oracle
 (tests/test_oracle_mutations.py) to show that each plausible mistake fails at
 least one of them.
@@ -284,7 +289,88 @@ def pin_dense_all_slots(so=None):
     np.testing.assert_allclose(out['o'], o, rtol=1e-6, atol=1e-6)
 
 
+# ---------------------------------------------------------------- near-tie flags
+# Score tables with n = 4 rows per half, k = 2, W = R = 2.  The key k' uses
+# coordinate 0 of each half and the query q' coordinate 1 (d_h = 2), so
+# C1[:, 0] / C2[:, 0] are the key's half-score tables and C1[:, 1] / C2[:, 1]
+# the query's, and each side's flags can be driven on its own.
+#
+# base: s1 = [3, 2, 0, -1], s2 = [3, 1, 0, -1].  Candidates of the top-2 rows:
+#   6, 5, 4, 3 -> the 2nd/3rd gap is 1/5; each half's rank-1/rank-2 gap is large.
+_FLAG_BASE = ([3.0, 2.0, 0.0, -1.0], [3.0, 1.0, 0.0, -1.0])
+
+
+def _flag_tables(case, delta):
+    """(s1, s2) of a side whose relative gap `delta` sits where `case` says:
+    'boundary': the 2nd/3rd candidate, 5 and 5 - 5 delta (bit 0 / 3);
+    'half1'   : half 1's k-th/(k+1)-th rows, 2 and 2 - 2 delta (bit 1 / 4);
+    'half2'   : half 2's k-th/(k+1)-th rows, 1 and 1 - delta (bit 2 / 5);
+    'rank01'  : half 1's 1st/2nd rows, 3 and 3 - 3 delta, which are not at
+                any selection boundary (no bit)."""
+    s1, s2 = list(_FLAG_BASE[0]), list(_FLAG_BASE[1])
+    if case == "boundary":
+        s2[1] = 2.0 - 5.0 * delta     # candidates 6, 5, 5 - 5 delta, 4 - 5 delta
+    elif case == "half1":
+        s1[2] = 2.0 - 2.0 * delta
+    elif case == "half2":
+        s2[2] = 1.0 - delta
+    elif case == "rank01":
+        s1[1] = 3.0 - 3.0 * delta     # candidates 6, 6 - 3 delta, 4, ...: 2nd/3rd far
+    return s1, s2
+
+
+_FLAG_BIT = {"boundary": 1, "half1": 2, "half2": 4, "rank01": 0}
+
+
+def pin_near_tie_flags(so=None):
+    d = _dims(T=1, d_qk=4, d_v=4, n_sub=4, k=2, W=2, R=2)
+    for side in ("key", "query"):
+        for case in ("boundary", "half1", "half2", "rank01"):
+            for delta, flagged in ((0.9e-5, True), (1.1e-5, False)):
+                t1, t2 = _flag_tables(case, delta)
+                b1, b2 = _FLAG_BASE
+                key1, key2 = (t1, t2) if side == "key" else (b1, b2)
+                qry1, qry2 = (t1, t2) if side == "query" else (b1, b2)
+                C1 = np.array([key1, qry1], np.float32).T[None]      # [1, n, 2]
+                C2 = np.array([key2, qry2], np.float32).T[None]
+                inp = dict(k=np.array([1, 0, 1, 0], np.float32)[None, None, None],
+                           q=np.array([0, 1, 0, 1], np.float32)[None, None, None],
+                           v=np.ones((1, 1, 1, 4), np.float32),
+                           alpha=np.ones((1, 1, 1), np.float32),
+                           beta=np.ones((1, 1, 1), np.float32), C1=C1, C2=C2,
+                           M0=np.zeros((1, 1, 16, 4), np.float32))
+                out = oracle.forward(inp, d, lists=True, so=so)
+                bit = _FLAG_BIT[case] if flagged else 0
+                expect = bit if side == "key" else bit << 3
+                got = int(out['flags'][0, 0, 0])
+                assert got == expect, (side, case, delta, got, expect)
+
+
+def pin_near_tie_flags_float64_gap(so=None):
+    """The flag reads the float64 gap, not the float32 one.  s1 = [1, 1 - g, -10],
+    s2 = [2^-24, -10, -20], x = [1, 1], W = 1, k = 2, g = 168 * 2^-24.  The best
+    candidate is 1 + 2^-24 exactly in float64, which rounds (to even) to 1.0 in
+    float32; the second is 1 - 167 * 2^-24 exactly in both.  The float64 gap,
+    168 * 2^-24 / (1 + 2^-24) = 1.0014e-5 relative, is above 1e-5 (no flag); the
+    float32 one, 167 * 2^-24 = 9.95e-6, would be below it."""
+    e = 2.0 ** -24
+    g = 168 * e
+    d = _dims(d_qk=2, n_sub=3, k=2, W=1, R=1)
+    C1 = np.array([[1.0], [1.0 - g], [-10.0]], np.float32)
+    C2 = np.array([[e], [-10.0], [-20.0]], np.float32)
+    assert float(C1[1, 0]) == 1.0 - g and float(C2[0, 0]) == e
+    assert np.float32(1.0) + np.float32(e) == np.float32(1.0)
+    slots, _, s, flag = oracle.select(np.array([1.0, 1.0], np.float32), C1, C2, d, 1, so=so)
+    assert int(slots[0]) == 0 and float(s[0]) == 1.0
+    assert flag == 0, flag
+    # the same tables with g = 167 * 2^-24: the float64 gap is below 1e-5
+    C1[1, 0] = np.float32(1.0 - 167 * e)
+    _, _, _, flag = oracle.select(np.array([1.0, 1.0], np.float32), C1, C2, d, 1, so=so)
+    assert flag == 1, flag
+
+
 ALL_PINS = [pin_golden, pin_bruteforce_identity, pin_gates_identity,
             pin_overwrite_and_read_after_write, pin_single_slot_recurrence, pin_softmax_weights,
             pin_ties_lowest_index, pin_half_split_and_slot_numbering, pin_untouched_rows,
-            pin_streaming, pin_dense_all_slots]
+            pin_streaming, pin_dense_all_slots, pin_near_tie_flags,
+            pin_near_tie_flags_float64_gap]

@@ -62,6 +62,23 @@ MUTANTS = {
     "read-before-write": _swap_read_write,
     "read-uses-write-weights": lambda s: s.replace(
         "acc[col] += rw[j] * (double)row[col];", "acc[col] += ww[j % d->W] * (double)row[col];"),
+    "near-tie-threshold-1e-3": lambda s: s.replace(
+        "return fabs(a - b) < 1e-5 * m;", "return fabs(a - b) < 1e-3 * m;"),
+    "near-tie-never-flagged": lambda s: s.replace(
+        "return fabs(a - b) < 1e-5 * m;", "return 0 * m * a * b;"),
+    "near-tie-on-float32-scores": lambda s: s.replace(
+        "near_tie(w->cand[n_sel - 1].s64, w->cand[n_sel].s64)",
+        "near_tie(w->cand[n_sel - 1].s, w->cand[n_sel].s)"),
+    "read-flags-not-shifted": lambda s: s.replace(
+        "select_side(io->q + (size_t)t * dq, io->C1, io->C2, d, d->R, &w, rs, rw, NULL, 3);",
+        "select_side(io->q + (size_t)t * dq, io->C1, io->C2, d, d->R, &w, rs, rw, NULL, 0);"),
+    "half-flags-swapped": lambda s: s.replace(
+        "flags |= 2 << flag_shift;", "flags |= 8 << flag_shift;").replace(
+        "flags |= 4 << flag_shift;", "flags |= 2 << flag_shift;").replace(
+        "flags |= 8 << flag_shift;", "flags |= 4 << flag_shift;"),
+    "half-flag-wrong-pair": lambda s: s.replace(
+        "near_tie(w->s64_1[w->h1[k - 1].id], w->s64_1[w->h1[k].id])",
+        "near_tie(w->s64_1[w->h1[k > 1 ? k - 2 : 0].id], w->s64_1[w->h1[k - 1].id])"),
     "fp64-candidate-order": lambda s: s.replace(
         "float s = w->h1[a].s + w->h2[b].s;          /* float32 sum */",
         "float s = (float)(w->s64_1[w->h1[a].id] + w->s64_2[w->h2[b].id]);"),
