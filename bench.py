@@ -9,14 +9,18 @@ selection, gated delta recurrence, reads) over the batch.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sdm|reference]
                   [--config 0..4] [--T steps] [--decode] [--probe-rows]
 
-Prints one JSON line (rank 0).  Under torchrun each rank runs its own shard of
-the batch (weak scaling, no collective on the data path); time is the max over
-ranks of the summed per-step CUDA-event times, with L2 flushed between steps.
-The line also carries: the roofline of the dominant kernel; the random-row
-ceiling of the recurrence's access pattern, measured in the same run; an
-end-to-end rate through the public API with pinned host inputs and outputs
-copied every step (pipelined with the compute, as a serving loop would); and
-the oracle timed on the host cores.  --impl reference times the oracle alone.
+Prints one JSON line (rank 0).  Under torchrun each rank owns a contiguous
+range of the flat (b,h) heads of a world-times-larger head grid (weak scaling,
+no collective on the data path) and runs it as rectangular pieces of the grid;
+time is the max over ranks of the summed per-step CUDA-event times, with L2
+flushed between steps.  The line also carries: the roofline of the dominant
+kernel and of the scoring contraction; the random-row ceiling of the
+recurrence's access pattern, measured in the same run; an end-to-end rate
+through the public API with pinned host inputs and outputs copied every step
+(pipelined with the compute, as a serving loop would); the oracle timed on the
+host cores (all of them, and one); and a parity sample: the GPU's selections
+against the oracle's on the oracle's sample, with the rate of near-ties the
+oracle flagged.  --impl reference times the oracle alone.
 """
 from __future__ import annotations
 
@@ -71,9 +75,9 @@ def peaks():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one k_recur
-# launch per token-head, from an ncu capture of the pages-scale workload at
-# T = 1024 (8192 token-heads; profiles/k_recur_dram_pages_scale_T1024.md),
-# valid for the recurrence source it was taken on.
+# launch per token-head, measured by ncu on the pages-scale workload at
+# T = 1024 (8192 token-heads): 270.9 MB read + 89.9 MB written.  Valid only for
+# the recurrence source it was taken on (its SHA-256 below).
 RECUR_DRAM_BYTES_PER_TOKEN_HEAD = (270892032 + 89945600) / 8192.0
 RECUR_DRAM_SOURCE_SHA256 = "ce6f96528744c2ecea01b7e144f1718abd36b675eaf6233e5709df5d3240523c"
 
@@ -159,8 +163,9 @@ class ClockSampler:
 # ----------------------------------------------------------------- cpu baseline
 def cpu_baseline(cfg, target_s: float, b0: int = 0):
     """The oracle, as it stands, on a bounded sample of the workload: the first
-    min(B*H, host threads) heads over a prefix of T_s steps."""
-    import numpy as np
+    min(B*H, host threads) heads over a prefix of T_s steps, on all host threads;
+    then one head on one thread.  Returns the baseline and the oracle's lists of
+    the sample (for the parity sample)."""
     import oracle
     from synth import gen_inputs
 
@@ -187,47 +192,96 @@ def cpu_baseline(cfg, target_s: float, b0: int = 0):
     dd = dict(Bs.dims(), T=T_s)
     flat = [b * cfg.H + h for b, h in heads]
     t = time.perf_counter()
-    oracle.forward(npi, dd, heads=flat, nthreads=nthr)
+    ref = oracle.forward(npi, dd, heads=flat, nthreads=nthr, lists=True)
     el = time.perf_counter() - t
-    return {"value": nheads * T_s / el, "unit": UNIT, "cores": min(nthr, nheads), "kind": "oracle",
+    # one head, one thread, a quarter of the time
+    T_1 = int(max(16, min(cfg.T, target_s / 4 / max(per_step, 1e-9))))
+    one = gen_inputs(sub, t_end=T_1, b0=b0)
+    t = time.perf_counter()
+    oracle.forward({k: v.numpy() for k, v in one.items()}, dict(cfg.dims(), B=1, H=1, T=T_1),
+                   nthreads=1)
+    el1 = time.perf_counter() - t
+    base = {"value": nheads * T_s / el, "unit": UNIT, "cores": min(nthr, nheads), "kind": "oracle",
             "sample": "%d heads x first %d steps of %s (oracle C, float64, %d threads, %.1f s)"
-                      % (nheads, T_s, cfg.name, min(nthr, nheads), el)}
+                      % (nheads, T_s, cfg.name, min(nthr, nheads), el),
+            "value_1thread": T_1 / el1,
+            "sample_1thread": "1 head x first %d steps, 1 thread, %.1f s" % (T_1, el1)}
+    return base, {"ref": ref, "heads": heads, "T": T_s}
+
+
+def parity_sample(lists, sample):
+    """GPU selections (sdm_select lists of the first batch rows) against the
+    oracle's on the CPU baseline's sample: mismatched sets, and how many of them
+    and of all selections the oracle flagged as near-ties."""
+    import numpy as np
+    ref, T = sample["ref"], sample["T"]
+    n_sel = mism = unflagged = flagged = 0
+    for (b, h) in sample["heads"]:
+        fl = ref["flags"][b, h, :T]
+        for gi, oi, bits in ((lists[0], ref["idx_w"], 0b000111), (lists[2], ref["idx_r"], 0b111000)):
+            g = np.sort(gi[b, h, :T].cpu().numpy().astype(np.int64), -1)
+            o = np.sort(oi[b, h, :T], -1)
+            same = (g == o).all(-1)
+            f = (fl & bits) != 0
+            n_sel += same.size
+            mism += int((~same).sum())
+            unflagged += int((~same & ~f).sum())
+            flagged += int(f.sum())
+    return {"selections": n_sel, "mismatched": mism, "unflagged_mismatched": unflagged,
+            "flagged_near_ties": flagged, "flagged_rate": flagged / max(1, n_sel),
+            "sample": "the CPU baseline's heads and steps"}
 
 
 # ---------------------------------------------------------------------- sdm arm
+def _device_uuid(torch, dev):
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        return None
+
+
 def run_sdm(args, cfg, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     import sparse_memory_linear_scoring_b200 as sdm
+    from sparse_memory_linear_scoring_b200.parallel import head_pieces, max_over_ranks, shard_heads
     from synth import gen_inputs
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    from sparse_memory_linear_scoring_b200.parallel import max_over_ranks, shard_batch
-    dims = sdm.make_dims(**cfg.dims())
-    plan = sdm.query_plan(dims)
-    # weak scaling: rank r owns batch rows [r*B, (r+1)*B) of a world*B batch
-    b0, _ = shard_batch(cfg.B * world, world, rank)
+    # weak scaling: the head grid is (world * B) x H; rank r owns the flat heads
+    # [r*B*H, (r+1)*B*H), run as rectangular pieces of the grid (here one piece
+    # of B batch rows, since B*H is a whole number of rows)
+    f0, nh = shard_heads(world * cfg.BH, world, rank)
+    pieces = head_pieces(f0, nh, cfg.H)
     dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
-    # inputs made on the device by the seeded generator, one batch row at a
-    # time (the high-batch table is 64 GiB)
-    d = {}
-    M = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d_v, dtype=torch.float32, device=dev)
-    for b in range(cfg.B):
-        part = gen_inputs(cfg.with_(B=1), device=str(dev), b0=b0 + b)
-        for n in ("q", "k", "v", "alpha", "beta"):
-            if n not in d:
-                shape = (cfg.B,) + tuple(part[n].shape[1:])
-                d[n] = torch.empty(shape, dtype=dt if n in ("q", "k", "v") else torch.float32,
-                                   device=dev)
-            d[n][b] = part[n][0]
-        M[b] = part["M0"][0]
-        if b == 0:
-            d["C1"] = part["C1"].to(dt).contiguous()
-            d["C2"] = part["C2"].to(dt).contiguous()
-        del part
-    o = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device=dev)
+    runs = []
+    for pc in pieces:
+        pcfg = cfg.with_(B=pc.b1 - pc.b0, H=pc.h1 - pc.h0)
+        # inputs made on the device by the seeded generator, one batch row at a
+        # time (the high-batch table is 64 GiB)
+        d = {}
+        M = torch.empty(pcfg.B, pcfg.H, cfg.N, cfg.d_v, dtype=torch.float32, device=dev)
+        for i in range(pcfg.B):
+            part = gen_inputs(cfg.with_(B=1), device=str(dev), b0=pc.b0 + i, h0=pc.h0, h1=pc.h1)
+            for n in ("q", "k", "v", "alpha", "beta"):
+                if n not in d:
+                    shape = (pcfg.B,) + tuple(part[n].shape[1:])
+                    d[n] = torch.empty(shape, dtype=dt if n in ("q", "k", "v") else torch.float32,
+                                       device=dev)
+                d[n][i] = part[n][0]
+            M[i] = part["M0"][0]
+            if i == 0:
+                d["C1"] = part["C1"].to(dt).contiguous()
+                d["C2"] = part["C2"].to(dt).contiguous()
+            del part
+        d["M"] = M
+        d["o"] = torch.empty(pcfg.B, pcfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device=dev)
+        runs.append((pcfg, d, sdm.query_plan(sdm.make_dims(**pcfg.dims()))))
+    plan = runs[0][2]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # phase events of the first piece (the only one unless heads split rows)
     nph = 5 * plan["chunks"]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(nph)]
     for e in ev:          # torch creates the CUDA event on its first record
@@ -235,8 +289,10 @@ def run_sdm(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize(dev)
 
     def step(events=None):
-        sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], M,
-                    topk=cfg.k, W=cfg.W, R=cfg.R, o=o, events=events)
+        for i, (pcfg, d, _) in enumerate(runs):
+            sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], d["M"],
+                        topk=cfg.k, W=cfg.W, R=cfg.R, o=d["o"],
+                        events=events if i == 0 else None)
 
     for _ in range(args.warmup):
         step()
@@ -245,13 +301,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
     if st != 0:
         raise RuntimeError("device status %d (info %d) after warm-up" % (st, info))
 
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-    except Exception:
-        uuid = None
-    clocks = ClockSampler(uuid)
+    clocks = ClockSampler(_device_uuid(torch, dev))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -289,17 +339,22 @@ def run_sdm(args, cfg, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         names = ("q", "k", "v", "alpha", "beta")
-        host = {n: torch.empty_like(d[n], device="cpu").pin_memory() for n in names}
-        for n in names:
-            host[n].copy_(d[n])
-        o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
-        dbuf = [{n: torch.empty_like(d[n]) for n in names} for _ in range(2)]
-        obuf = [torch.empty_like(o) for _ in range(2)]
-        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-        d2h = o_host[0].numel() * o_host[0].element_size()
         comp = torch.cuda.current_stream(dev)
         cin = torch.cuda.Stream(dev)
         cout = torch.cuda.Stream(dev)
+        pipes = []
+        h2d = d2h = 0
+        for pcfg, d, _ in runs:
+            host = {n: torch.empty_like(d[n], device="cpu").pin_memory() for n in names}
+            for n in names:
+                host[n].copy_(d[n])
+            o_host = [torch.empty(d["o"].shape, dtype=d["o"].dtype).pin_memory()
+                      for _ in range(2)]
+            dbuf = [{n: torch.empty_like(d[n]) for n in names} for _ in range(2)]
+            obuf = [torch.empty_like(d["o"]) for _ in range(2)]
+            h2d += sum(host[n].numel() * host[n].element_size() for n in names)
+            d2h += o_host[0].numel() * o_host[0].element_size()
+            pipes.append((d, host, o_host, dbuf, obuf))
 
         def run_pipeline(nsteps, start=None):
             if start is not None:
@@ -312,19 +367,22 @@ def run_sdm(args, cfg, rank, world, local_rank):
                 with torch.cuda.stream(cin):
                     if i >= 2:
                         cin.wait_event(ev_done[i - 2])   # buffer j is free again
-                    for n in names:
-                        dbuf[j][n].copy_(host[n], non_blocking=True)
+                    for (_, host, _, dbuf, _) in pipes:
+                        for n in names:
+                            dbuf[j][n].copy_(host[n], non_blocking=True)
                     ev_in[i].record(cin)
                 comp.wait_event(ev_in[i])
                 if i >= 2:
                     comp.wait_event(ev_out[i - 2])       # o buffer j was copied out
-                sdm.forward(dbuf[j]["q"], dbuf[j]["k"], dbuf[j]["v"], dbuf[j]["alpha"],
-                            dbuf[j]["beta"], d["C1"], d["C2"], M, topk=cfg.k, W=cfg.W, R=cfg.R,
-                            o=obuf[j])
+                for (d, _, _, dbuf, obuf) in pipes:
+                    sdm.forward(dbuf[j]["q"], dbuf[j]["k"], dbuf[j]["v"], dbuf[j]["alpha"],
+                                dbuf[j]["beta"], d["C1"], d["C2"], d["M"], topk=cfg.k, W=cfg.W,
+                                R=cfg.R, o=obuf[j])
                 ev_done[i].record(comp)
                 with torch.cuda.stream(cout):
                     cout.wait_event(ev_done[i])
-                    o_host[j].copy_(obuf[j], non_blocking=True)
+                    for (_, _, o_host, _, obuf) in pipes:
+                        o_host[j].copy_(obuf[j], non_blocking=True)
                     ev_out[i].record(cout)
             comp.wait_stream(cout)
             comp.wait_stream(cin)
@@ -344,7 +402,16 @@ def run_sdm(args, cfg, rank, world, local_rank):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": et / args.steps,
                "pipelined": "copies of steps i+1 (in) and i-1 (out) overlap step i",
-               "l2": "not flushed: the 2 GiB state is larger than L2"}
+               "l2": "not flushed: the state is larger than L2"}
+        del pipes
+
+    # the selection lists of the first piece, for the parity sample
+    lists = None
+    if rank == 0 and not args.no_cpu_baseline:
+        pcfg, d, _ = runs[0]
+        lists = sdm.select(d["q"], d["k"], d["C1"], d["C2"], topk=cfg.k, W=cfg.W, R=cfg.R,
+                           d_v=cfg.d_v)
+        torch.cuda.synchronize(dev)
 
     # the random-row ceiling of the recurrence's access pattern, this run
     pat = None
@@ -352,7 +419,7 @@ def run_sdm(args, cfg, rank, world, local_rank):
         del flush
         pat = pattern_ceiling(cfg.W, cfg.R)
     if rank != 0:
-        return None
+        return None, None
     pk, src = peaks()
     K = args.steps
     th = cfg.BH * cfg.T
@@ -361,35 +428,46 @@ def run_sdm(args, cfg, rank, world, local_rank):
     shares = {n: phase[i] / max(1e-12, sum(phase)) for i, n in enumerate(names)}
     per = {n: phase[i] / K for i, n in enumerate(names)}
     dom = max(names, key=lambda n: per[n])
-    slot_bytes = th * (2 * cfg.W + cfg.R) * cfg.d_v * 4
-    score_flops = th * 4 * cfg.n_sub * cfg.d_qk
-    if dom == "recur":
-        roof = {"kernel": "k_recur", "bound": "hbm",
-                "achieved": slot_bytes / (per["recur"] / 1e3) / 1e9,
-                "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    elif dom == "score" and plan["tensor_core_scoring"]:
-        roof = {"kernel": "k_score_tc", "bound": "tensor",
-                "achieved": score_flops / (per["score"] / 1e3) / 1e12,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
-    else:
-        # CUDA-core kernels: float32 FMA peak = 148 SMs x 128 lanes x 2 x max clock
-        fp32_peak = 148 * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
-        kname = {"score": "k_score_simt", "merge": "k_merge", "plan": "k_plan"}[dom]
-        roof = {"kernel": kname, "bound": "alu",
-                "achieved": (score_flops / (per[dom] / 1e3) / 1e12) if dom == "score" else None,
-                "peak": fp32_peak, "unit": "TFLOP/s"}
-    roof["frac"] = (roof["achieved"] / roof["peak"]) if roof["achieved"] else None
-    roof["traffic"] = recur_traffic(th) if roof["kernel"] == "k_recur" else None
-    roof["peak_source"] = src
+    th0 = runs[0][0].BH * cfg.T                 # token-heads of the timed piece
+    slot_bytes = th0 * (2 * cfg.W + cfg.R) * cfg.d_v * 4
+    score_flops = th0 * 4 * cfg.n_sub * cfg.d_qk
+    fp32_peak = 148 * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
     rec_gbs = slot_bytes / (per["recur"] / 1e3) / 1e9
+    if plan["tensor_core_scoring"]:
+        roof_s = {"kernel": "k_score_tc", "bound": "tensor",
+                  "achieved": score_flops / (per["score"] / 1e3) / 1e12,
+                  "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "peak_kind": "bf16 burst"}
+    else:
+        roof_s = {"kernel": "k_score_warp", "bound": "alu",
+                  "achieved": score_flops / (per["score"] / 1e3) / 1e12,
+                  "peak": fp32_peak, "unit": "TFLOP/s",
+                  "peak_kind": "float32 FMA, 148 SMs x 128 lanes x 2 x max clock"}
+    roof_s["frac"] = roof_s["achieved"] / roof_s["peak"]
+    roof_s["flops_per_launch"] = score_flops
+    roof_s["peak_source"] = src
+    if dom == "recur":
+        roof = {"kernel": "k_recur", "bound": "hbm", "achieved": rec_gbs,
+                "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "traffic": recur_traffic(th0) if plan["chunks"] == 1 else None,
+                "bytes_per_launch": slot_bytes / plan["chunks"]}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+    elif dom == "score":
+        roof = dict(roof_s, traffic=None)
+    else:
+        roof = {"kernel": {"merge": "k_merge", "plan": "k_plan"}[dom], "bound": "alu",
+                "achieved": None, "peak": fp32_peak, "unit": "TFLOP/s", "frac": None,
+                "traffic": None}
+    roof["peak_source"] = src
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": t_max / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world,
-                   "heads": cfg.H, "seq_len": cfg.T, "parallelism": "dp%d (heads sharded, no collective)" % world,
+                   "heads": cfg.H, "seq_len": cfg.T,
+                   "parallelism": "dp%d: (b,h) heads sharded across ranks, no collective" % world,
                    "l2": "flushed between steps (256 MiB write)"},
         "roofline": roof,
+        "roofline_scoring": roof_s,
         "slot_traffic": {"bytes_per_step": slot_bytes, "recur_gbs": rec_gbs,
                          "recur_frac_of_8TBs": rec_gbs / 8000.0,
                          "recur_frac_of_measured": rec_gbs / pk["hbm_gbs"],
@@ -398,10 +476,10 @@ def run_sdm(args, cfg, rank, world, local_rank):
                          "recur_frac_of_pattern_ceiling":
                              rec_gbs / pat["ceiling_gbs"] if pat else None},
         "phases_ms": per, "phase_share": shares, "plan": plan,
-        "gpu_launches": int(plan["launches_per_call"] * K),
+        "gpu_launches": int(sum(r[2]["launches_per_call"] for r in runs) * K),
         "clocks": clk, "e2e": e2e,
     }
-    return out
+    return out, lists
 
 
 # ---------------------------------------------------------------- reference arm
@@ -450,7 +528,7 @@ def probe_rows(configs=None):
     """Random whole-row gathers / read-modify-writes on a 2 GiB table (the size of
     the pages-scale slot tables), timed with CUDA events after a warm-up launch."""
     import torch
-    import sparse_memory_linear_scoring_b200 as sdm
+    from sparse_memory_linear_scoring_b200.probe import probe_random_rows
     nrows = 8 << 20
     table = torch.zeros(nrows, 64, dtype=torch.float32, device="cuda")
     res = []
@@ -461,11 +539,11 @@ def probe_rows(configs=None):
         if True:
             if True:
                 iters = 64
-                sdm.probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=4)
+                probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=4)
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record()
-                sdm.probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=iters)
+                probe_random_rows(table, rmw=rmw, rows_in_flight=u, ctas=ctas, iters=iters)
                 e1.record()
                 e1.synchronize()
                 ms = e0.elapsed_time(e1)
@@ -575,10 +653,12 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    out = run_sdm(args, cfg, rank, world, local_rank)
+    out, lists = run_sdm(args, cfg, rank, world, local_rank)
     if rank == 0:
         if not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
+            out["cpu_baseline"], sample = cpu_baseline(cfg, args.cpu_seconds)
+            if lists is not None:
+                out["parity_sample"] = parity_sample(lists, sample)
         print(json.dumps(out), flush=True)
     if world > 1:
         import torch.distributed as dist

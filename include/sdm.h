@@ -203,20 +203,6 @@ SDM_API int sdm_get_device_status(const void* workspace, size_t ws_bytes, int32_
 /* Static text for a return code (never NULL). */
 SDM_API const char* sdm_status_string(int status);
 
-/*
- * Measurement helper, not part of the method: launches `ctas` CTAs of 256
- * threads that each move, per iteration, rows_in_flight (4 or 8) random whole
- * rows of 64 floats (256 bytes) per group of 8 threads in `table` (nrows rows,
- * device memory, 16-byte aligned): loads only (rmw = 0) or load, add and store
- * back (rmw = 1), `iters` times.  Bytes moved = ctas * 32 * rows_in_flight *
- * iters * 256 (times 2 with rmw).  It gives the HBM ceiling of the
- * recurrence's random-row access pattern.  Asynchronous on `stream`; the table
- * is modified when rmw = 1.  Returns SDM_OK, SDM_ERR_NULL, SDM_ERR_DIMS,
- * SDM_ERR_ALIGN, SDM_ERR_UNSUPPORTED or SDM_ERR_CUDA.
- */
-SDM_API int sdm_probe_random_rows(float* table, long long nrows, int rmw, int rows_in_flight,
-                                  int ctas, int iters, void* stream);
-
 /* Library version, major*10000 + minor*100 + patch. */
 SDM_API int sdm_version(void);
 

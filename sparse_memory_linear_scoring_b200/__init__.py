@@ -8,5 +8,5 @@ without the built library, or with CPU tensors, raises.
 """
 from .sdm import (  # noqa: F401
     SDMError, Dims, LIB_PATH, load_library, workspace_bytes, forward, select, recur,
-    device_status, make_dims, query_plan, PLAN_FIELDS, probe_random_rows,
+    device_status, make_dims, query_plan, PLAN_FIELDS,
 )

@@ -1,11 +1,22 @@
-// probe_rows.cu -- measurement helper: the HBM bandwidth of the recurrence's
-// access pattern on its own, i.e. random whole-row (256-byte) gathers and
-// read-modify-writes of a float32 table, with many rows in flight.  It gives
-// the pattern's practical ceiling beside the streaming-copy peak.
-#include "sdm_internal.cuh"
+// probe_rows.cu -- measurement helper, built into its own library
+// (libsdm_probe.so) and not part of the SDM C ABI: the HBM bandwidth of the
+// recurrence's access pattern on its own, i.e. random whole-row (256-byte)
+// gathers and read-modify-writes of a float32 table, with many rows in flight.
+// It gives the pattern's practical ceiling beside the streaming-copy peak.
+#include <cuda_runtime.h>
+#include <stdint.h>
 
-namespace sdm {
+#include "probe_rows.h"
+
+namespace sdm_probe {
 namespace {
+
+__device__ __forceinline__ uint32_t hash32(uint32_t x) {
+  x ^= x >> 16; x *= 0x7feb352du;
+  x ^= x >> 15; x *= 0x846ca68bu;
+  x ^= x >> 16;
+  return x;
+}
 
 // 8 lanes per 64-float row, 32 bytes per lane; U rows in flight per lane group
 template <int U, bool RMW>
@@ -17,7 +28,7 @@ __global__ void __launch_bounds__(256) k_probe_rows(float* __restrict__ M, long 
     float4 a[U], b[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      r[u] = (long long)(mix32(uint32_t(g) * 7919u + uint32_t(it * U + u) ^ seed) %
+      r[u] = (long long)(hash32(uint32_t(g) * 7919u + uint32_t(it * U + u) ^ seed) %
                          uint32_t(nrows));
       const float* ptr = M + r[u] * 64 + l * 8;
       asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
@@ -46,15 +57,15 @@ __global__ void __launch_bounds__(256) k_probe_rows(float* __restrict__ M, long 
 }
 
 }  // namespace
-}  // namespace sdm
+}  // namespace sdm_probe
 
-using namespace sdm;
+using namespace sdm_probe;
 
-extern "C" int sdm_probe_random_rows(float* table, long long nrows, int rmw, int rows_in_flight,
+extern "C" SDM_PROBE_API int sdm_probe_random_rows(float* table, long long nrows, int rmw, int rows_in_flight,
                                      int ctas, int iters, void* stream) {
-  if (!table) return SDM_ERR_NULL;
-  if (nrows < 1 || nrows > 0xffffffffLL || ctas < 1 || iters < 1) return SDM_ERR_DIMS;
-  if (reinterpret_cast<uintptr_t>(table) & 15) return SDM_ERR_ALIGN;
+  if (!table) return SDM_PROBE_ERR_NULL;
+  if (nrows < 1 || nrows > 0xffffffffLL || ctas < 1 || iters < 1) return SDM_PROBE_ERR_DIMS;
+  if (reinterpret_cast<uintptr_t>(table) & 15) return SDM_PROBE_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint32_t seed = 0x5bd1e995u;
   if (rows_in_flight == 4) {
@@ -64,7 +75,7 @@ extern "C" int sdm_probe_random_rows(float* table, long long nrows, int rmw, int
     if (rmw) k_probe_rows<8, true><<<ctas, 256, 0, s>>>(table, nrows, iters, seed);
     else k_probe_rows<8, false><<<ctas, 256, 0, s>>>(table, nrows, iters, seed);
   } else {
-    return SDM_ERR_UNSUPPORTED;
+    return SDM_PROBE_ERR_UNSUPPORTED;
   }
-  return cudaGetLastError() == cudaSuccess ? SDM_OK : SDM_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? SDM_PROBE_OK : SDM_PROBE_ERR_CUDA;
 }

@@ -301,16 +301,3 @@ def device_status(workspace: Optional[torch.Tensor] = None, stream=None) -> Tupl
                                                 ctypes.byref(st), ctypes.byref(info),
                                                 _stream(workspace.device, stream)))
     return int(st.value), int(info.value)
-
-
-def probe_random_rows(table: torch.Tensor, *, rmw: bool, rows_in_flight: int, ctas: int,
-                      iters: int, stream=None) -> None:
-    """Measurement helper (sdm_probe_random_rows): random whole-row gathers
-    (rmw=False) or read-modify-writes (rmw=True) of a float32 [nrows, 64] table."""
-    dev = _dev(table)
-    if table.dtype != torch.float32 or table.dim() != 2 or table.shape[1] != 64 or \
-            not table.is_contiguous():
-        raise ValueError("table must be a contiguous float32 [nrows, 64] CUDA tensor")
-    _check(load_library().sdm_probe_random_rows(_ptr(table), ctypes.c_longlong(table.shape[0]),
-                                                int(bool(rmw)), int(rows_in_flight), int(ctas),
-                                                int(iters), _stream(dev, stream)))

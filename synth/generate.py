@@ -193,11 +193,14 @@ def gen_head_inputs(cfg: SDMConfig, b: int, h: int, seed: int = 0,
 
 def gen_inputs(cfg: SDMConfig, seed: int = 0, device: str = 'cpu',
                t_end: Optional[int] = None, with_m0: bool = True,
-               b0: int = 0) -> Dict[str, torch.Tensor]:
+               b0: int = 0, h0: int = 0, h1: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """All inputs, full layout: q,k [B,H,T,d_qk], v [B,H,T,d_v], alpha,beta [B,H,T],
     C1,C2 [H,n,d_h], M0 [B,H,N,d_v] (float32 values).  b0 offsets the batch
-    index (a shard [b0, b0+B) of a larger batch)."""
-    return _gen(cfg, list(range(b0, b0 + cfg.B)), list(range(cfg.H)), seed, device, t_end,
+    index (rows [b0, b0+B) of a larger batch); h0, h1 select the heads [h0, h1)
+    of the cfg.H heads (default all), so that a rectangle of the head grid is
+    the same slice of the full inputs."""
+    h1 = cfg.H if h1 is None else h1
+    return _gen(cfg, list(range(b0, b0 + cfg.B)), list(range(h0, h1)), seed, device, t_end,
                 with_m0, squeeze=False)
 
 

@@ -40,8 +40,8 @@ def _check_forward(cfg, inp, ref, d=None):
     _, same_r = compare_lists(ir.cpu().numpy(), wr.cpu().numpy(), ref["idx_r"], ref["w_r"],
                               ref["flags"], READ_BITS, "read lists")
     clean = same_w.all(axis=-1) & same_r.all(axis=-1)          # [B,H]
-    eo = head_rel_err(o.cpu().numpy(), ref["o"])
-    eM = head_rel_err(M.cpu().numpy(), ref["M"])
+    eo = head_rel_err(o.cpu().numpy(), ref["o"], "o %s" % cfg.name)
+    eM = head_rel_err(M.cpu().numpy(), ref["M"], "M %s" % cfg.name)
     assert (eo[clean] <= REL_TOL).all(), eo
     assert (eM[clean] <= REL_TOL).all(), eM
     # the recurrence alone, fed the oracle's lists
@@ -194,17 +194,19 @@ def test_recur_flags_bad_lists():
 
 
 def test_probe_random_rows():
-    """The random-row bandwidth probe: gathers leave the table unchanged,
-    read-modify-writes add to it; bad arguments are rejected."""
+    """The benchmark's random-row bandwidth probe (its own library): gathers
+    leave the table unchanged, read-modify-writes add to it; bad arguments are
+    rejected."""
+    from sparse_memory_linear_scoring_b200.probe import probe_random_rows
     table = torch.zeros(4096, 64, dtype=torch.float32, device="cuda")
-    sdm.probe_random_rows(table, rmw=False, rows_in_flight=4, ctas=2, iters=2)
+    probe_random_rows(table, rmw=False, rows_in_flight=4, ctas=2, iters=2)
     torch.cuda.synchronize()
     assert int((table != 0).sum()) == 0
-    sdm.probe_random_rows(table, rmw=True, rows_in_flight=8, ctas=2, iters=2)
+    probe_random_rows(table, rmw=True, rows_in_flight=8, ctas=2, iters=2)
     torch.cuda.synchronize()
     assert float(table.sum()) > 0
-    with pytest.raises(sdm.SDMError):
-        sdm.probe_random_rows(table, rmw=True, rows_in_flight=3, ctas=2, iters=2)
+    with pytest.raises(ValueError):
+        probe_random_rows(table, rmw=True, rows_in_flight=3, ctas=2, iters=2)
 
 
 def _repeat_inputs(cfg, period, share_qk):

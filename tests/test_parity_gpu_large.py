@@ -4,18 +4,27 @@ M_0 ~ N(0, 0.02^2), 64 GiB table) workloads, in the launch configuration the
 benchmark uses (one forward call over the whole batch).
 
 The inputs are generated on the GPU by the seeded counter-based generator; the
-heads the oracle checks are copied back, so both sides see the same bytes.
-Checked: sampled selections against the oracle's selection (same sets except
-at flagged near-ties, weights within 2e-5), o over a prefix (long-context) or
-whole sampled heads (high-batch) within 1e-4 of the head's largest |o|, and
-rows never written staying bit-identical to M_0."""
+heads the oracle checks are copied back, so both sides see the same bytes.  The
+oracle runs those heads over the whole sequence, on host threads, while the GPU
+works.  Checked per head, against the oracle:
+  * every step's write and read sets equal, except at near-ties the oracle
+    flagged (at most 0.1% of selections); weights within 2e-5;
+  * every o_t and the final table M_T within 1e-4 of the head's largest |o|,
+    |M| -- from sdm_forward when the head's selections all agree, else from
+    sdm_recur fed the oracle's own lists (a legitimate tie flip would otherwise
+    be scored as numeric error from that step on);
+  * rows never written stay bit-identical to M_0.
+Long-context: 4 heads x 65,536 steps (about 5 minutes of oracle time on 4
+threads).  High-batch: 16 heads spread over b and h, 4,096 steps each."""
+import threading
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import sparse_memory_linear_scoring_b200 as sdm
-from gpu_util import READ_BITS, REL_TOL, W_TOL, WRITE_BITS
+from gpu_util import READ_BITS, REL_TOL, WRITE_BITS, compare_lists, elem_rel_err, ncpu, report
 from synth import config, gen_inputs
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -26,44 +35,88 @@ def _status_clean():
     assert st == 0, "device status %d (info %d)" % (st, info)
 
 
-def _head(d, b, h, t_end=None, M0=None):
-    """One head's inputs as float32 numpy arrays (exact copies of the device bytes)."""
-    sl = slice(0, t_end)
+def _packed_heads(d, heads, M0=None):
+    """The chosen (b,h) heads as one B=1, H=len(heads) problem of float32 numpy
+    arrays (exact copies of the device bytes), for the oracle."""
     out = {}
     for name in ("q", "k", "v", "alpha", "beta"):
-        out[name] = d[name][b, h, sl].float().cpu().numpy()
+        out[name] = torch.stack([d[name][b, h] for b, h in heads]).float().cpu().numpy()[None]
     for name in ("C1", "C2"):
-        out[name] = d[name][h].float().cpu().numpy()
+        out[name] = torch.stack([d[name][h] for _, h in heads]).float().cpu().numpy()
     out["M0"] = M0
     return out
 
 
-def _check_sampled_selections(cfg, hin, lists, b, h, steps):
-    """GPU lists at the sampled steps against oracle.select; returns mismatches."""
-    mism = 0
-    for t in steps:
-        for (x, gi, gw, n_sel) in ((hin["k"][t], lists[0], lists[1], cfg.W),
-                                   (hin["q"][t], lists[2], lists[3], cfg.R)):
-            slots, w, _, flag = oracle.select(x, hin["C1"], hin["C2"], cfg.dims(), n_sel)
-            g_s = gi[b, h, t].cpu().numpy().astype(np.int64)
-            g_w = gw[b, h, t].cpu().numpy().astype(np.float64)
-            if not np.array_equal(np.sort(g_s), np.sort(slots)):
-                assert flag & 0b111, "unflagged selection mismatch at (%d,%d,%d)" % (b, h, t)
-                mism += 1
-                continue
-            assert np.abs(g_w[np.argsort(g_s)] - w[np.argsort(slots)]).max() <= W_TOL
-    return mism
+class _OracleThread(threading.Thread):
+    """oracle.forward on host threads, started before the GPU work."""
+
+    def __init__(self, inp, dims):
+        super().__init__(daemon=True)
+        self.inp, self.dims, self.res, self.err = inp, dims, None, None
+
+    def run(self):
+        try:
+            self.res = oracle.forward(self.inp, self.dims, lists=True,
+                                      nthreads=max(1, min(ncpu(), self.dims["H"])))
+        except Exception as e:  # reported by the test
+            self.err = e
 
 
-def _same_sets(g_idx, o_idx):
-    return (np.sort(g_idx, -1) == np.sort(o_idx, -1)).all(-1)
+def _check_heads(cfg, d, heads, ref, o, M, lists, M0s):
+    """Per-head parity of the GPU outputs against the oracle's run of the heads."""
+    rel = lambda g, r: np.abs(g - r).max() / max(1e-30, np.abs(r).max())
+    for j, (b, h) in enumerate(heads):
+        g_iw = lists[0][b, h].cpu().numpy()
+        g_ir = lists[2][b, h].cpu().numpy()
+        _, same_w = compare_lists(g_iw, lists[1][b, h].cpu().numpy(), ref["idx_w"][0, j],
+                                  ref["w_w"][0, j], ref["flags"][0, j], WRITE_BITS,
+                                  "write lists (%d,%d)" % (b, h))
+        _, same_r = compare_lists(g_ir, lists[3][b, h].cpu().numpy(), ref["idx_r"][0, j],
+                                  ref["w_r"][0, j], ref["flags"][0, j], READ_BITS,
+                                  "read lists (%d,%d)" % (b, h))
+        r_o = ref["o"][0, j].astype(np.float64)
+        r_M = ref["M"][0, j].astype(np.float64)
+        if same_w.all() and same_r.all():
+            g_o = o[b, h].cpu().numpy().astype(np.float64)
+            g_M = M[b, h].cpu().numpy().astype(np.float64)
+        else:
+            # the recurrence alone on this head, fed the oracle's lists
+            sl = lambda t: t[b:b + 1, h:h + 1].contiguous()
+            cu = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a[None, None])).to(
+                device="cuda", dtype=dt)
+            Mh = torch.from_numpy(M0s[j]).cuda()[None, None].contiguous()
+            oh = sdm.recur(sl(d["v"]), sl(d["alpha"]), sl(d["beta"]),
+                           cu(ref["idx_w"][0, j], torch.int32), cu(ref["w_w"][0, j], torch.float32),
+                           cu(ref["idx_r"][0, j], torch.int32), cu(ref["w_r"][0, j], torch.float32),
+                           Mh, d_qk=cfg.d_qk, n_sub=cfg.n_sub, topk=cfg.k)
+            torch.cuda.synchronize()
+            _status_clean()
+            g_o = oh[0, 0].cpu().numpy().astype(np.float64)
+            g_M = Mh[0, 0].cpu().numpy().astype(np.float64)
+        for name, g, r in (("o", g_o, r_o), ("M", g_M, r_M)):
+            report("%s %s head (%d,%d)" % (name, cfg.name, b, h), rel(g, r),
+                   elem_rel_err(g[None, None], r[None, None]))
+        assert rel(g_o, r_o) <= REL_TOL, ("o", b, h, rel(g_o, r_o))
+        assert rel(g_M, r_M) <= REL_TOL, ("M", b, h, rel(g_M, r_M))
+        # rows never written keep M_0 exactly (GPU lists of the forward call)
+        untouched = np.ones(cfg.N, dtype=bool)
+        untouched[np.unique(g_iw)] = False
+        gM = M[b, h].cpu().numpy()
+        assert np.array_equal(gM[untouched], M0s[j][untouched])
 
 
-def test_long_context_full_size():
+def test_long_context_full_length():
     cfg = config(3)
     d = gen_inputs(cfg, device="cuda", with_m0=False)
     for name in ("q", "k", "v", "C1", "C2"):
         d[name] = d[name].to(torch.bfloat16).contiguous()
+    assert sdm.query_plan(sdm.make_dims(**cfg.dims()))["chunks"] >= 1
+    heads = [(0, 1), (0, 3), (0, 5), (0, 6)] if ncpu() >= 4 else [(0, 1), (0, 6)]
+    M0s = [np.zeros((cfg.N, cfg.d_v), np.float32) for _ in heads]
+    th = _OracleThread(_packed_heads(d, heads, np.zeros((1, len(heads), cfg.N, cfg.d_v),
+                                                        np.float32)),
+                       dict(cfg.dims(), B=1, H=len(heads)))
+    th.start()
     M = torch.zeros(cfg.B, cfg.H, cfg.N, cfg.d_v, dtype=torch.float32, device="cuda")
     o = sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], M,
                     topk=cfg.k, W=cfg.W, R=cfg.R)
@@ -73,41 +126,12 @@ def test_long_context_full_size():
                        d_v=cfg.d_v)
     torch.cuda.synchronize()
     _status_clean()
-
-    # selections at sampled steps of two heads: in the patterned half, at the
-    # boundary where the keys turn i.i.d., and in the i.i.d. half
-    rng = np.random.default_rng(3)
-    steps = sorted(set(rng.integers(0, cfg.T, 20).tolist())
-                   | {0, cfg.pattern_until - 1, cfg.pattern_until, cfg.T - 1})
-    mism = 0
-    for h in (1, 6):
-        hin = _head(d, 0, h)
-        mism += _check_sampled_selections(cfg, hin, lists, 0, h, steps)
-    assert mism <= 2
-
-    # o over a prefix, against the oracle run on that prefix
-    T_pre = 512
-    for h in (2, 5):
-        hin = _head(d, 0, h, T_pre, np.zeros((cfg.N, cfg.d_v), np.float32))
-        ref = oracle.forward_head(hin, cfg.dims(), lists=True)
-        same = _same_sets(lists[0][0, h, :T_pre].cpu().numpy(), ref["idx_w"]) & \
-            _same_sets(lists[2][0, h, :T_pre].cpu().numpy(), ref["idx_r"])
-        assert (ref["flags"][~same] != 0).all(), "unflagged selection mismatch"
-        upto = T_pre if same.all() else int(np.argmin(same))
-        assert upto >= T_pre // 4
-        g = o[0, h, :upto].cpu().numpy().astype(np.float64)
-        r = ref["o"][:upto].astype(np.float64)
-        assert np.abs(g - r).max() <= REL_TOL * np.abs(r).max()
-
-    # rows never written keep M_0 = 0 exactly; written rows are not all zero
-    for h in (0, 7):
-        written = torch.zeros(cfg.N, dtype=torch.bool, device="cuda")
-        written[lists[0][0, h].reshape(-1).long()] = True
-        assert int((M[0, h][~written] != 0).sum()) == 0
-        assert int((M[0, h][written].abs().sum(-1) > 0).sum()) > 0.99 * int(written.sum())
+    th.join()
+    assert th.err is None, th.err
+    _check_heads(cfg, d, heads, th.res, o, M, lists, M0s)
 
 
-def test_high_batch_full_size():
+def test_high_batch_16_heads():
     cfg = config(4)
     dt = torch.bfloat16
     dev = "cuda"
@@ -126,31 +150,17 @@ def test_high_batch_full_size():
         C2 = part["C2"].to(dt).contiguous()
         del part
     d = dict(q=q, k=k, v=v, alpha=al, beta=be, C1=C1, C2=C2)
-    sampled = [(0, 0), (17, 5), (40, 9), (63, 15)]
-    M0s = {bh: M[bh[0], bh[1]].cpu().numpy() for bh in sampled}
+    heads = [(4 * i + (i % 3), i) for i in range(16)]       # 16 batch rows, all 16 heads
+    M0s = [M[b, h].cpu().numpy() for b, h in heads]
+    th = _OracleThread(_packed_heads(d, heads, np.stack(M0s)[None]),
+                       dict(cfg.dims(), B=1, H=len(heads)))
+    th.start()
     o = sdm.forward(q, k, v, al, be, C1, C2, M, topk=cfg.k, W=cfg.W, R=cfg.R)
     torch.cuda.synchronize()
     _status_clean()
     lists = sdm.select(q, k, C1, C2, topk=cfg.k, W=cfg.W, R=cfg.R, d_v=cfg.d_v)
     torch.cuda.synchronize()
     _status_clean()
-    checked = 0
-    for (b, h) in sampled:
-        hin = _head(d, b, h, None, M0s[(b, h)])
-        ref = oracle.forward_head(hin, cfg.dims(), lists=True)
-        g_iw = lists[0][b, h].cpu().numpy().astype(np.int64)
-        g_ir = lists[2][b, h].cpu().numpy().astype(np.int64)
-        same = _same_sets(g_iw, ref["idx_w"]) & _same_sets(g_ir, ref["idx_r"])
-        assert (ref["flags"][~same] != 0).all(), "unflagged selection mismatch"
-        assert (~same).sum() <= 0.001 * cfg.T
-        if not same.all():
-            continue
-        go = o[b, h].cpu().numpy().astype(np.float64)
-        gM = M[b, h].cpu().numpy().astype(np.float64)
-        assert np.abs(go - ref["o"]).max() <= REL_TOL * np.abs(ref["o"]).max()
-        assert np.abs(gM - ref["M"]).max() <= REL_TOL * np.abs(ref["M"]).max()
-        untouched = np.ones(cfg.N, dtype=bool)
-        untouched[np.unique(g_iw)] = False
-        assert np.array_equal(gM[untouched].astype(np.float32), M0s[(b, h)][untouched])
-        checked += 1
-    assert checked >= 2
+    th.join()
+    assert th.err is None, th.err
+    _check_heads(cfg, d, heads, th.res, o, M, lists, M0s)
