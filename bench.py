@@ -569,8 +569,10 @@ def pattern_ceiling(W, R):
 
 
 def decode(cfg, steps):
-    """Streaming use: one sdm_forward call per step (T = 1) with M carried, on
-    the workload's B x H heads; eager launches and one CUDA graph of all steps."""
+    """Streaming use, M carried from call to call, on the workload's B x H heads:
+    one sdm_step call per step (the fused single-step kernel) and, for
+    comparison, one sdm_forward call per step (T = 1); each eager and as one
+    CUDA graph of all steps."""
     import torch
     import sparse_memory_linear_scoring_b200 as sdm
     from synth import gen_inputs
@@ -587,43 +589,52 @@ def decode(cfg, steps):
     ws = torch.empty(sdm.workspace_bytes(dims), dtype=torch.uint8, device="cuda")
     o = torch.empty(steps, cfg.B, cfg.H, 1, cfg.d_v, dtype=torch.float32, device="cuda")
 
-    def one(t):
+    def one_forward(t):
         a = per["alpha"][t].squeeze(-1)
         b = per["beta"][t].squeeze(-1)
         sdm.forward(per["q"][t], per["k"][t], per["v"][t], a, b, C1, C2, M, topk=cfg.k,
                     W=cfg.W, R=cfg.R, o=o[t], workspace=ws)
 
-    for t in range(min(steps, 8)):
-        one(t)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for t in range(steps):
-        one(t)
-    e1.record()
-    e1.synchronize()
-    eager_us = e0.elapsed_time(e1) * 1e3 / steps
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g, stream=s):
-            for t in range(steps):
-                one(t)
-    torch.cuda.current_stream().wait_stream(s)
-    g.replay()
-    torch.cuda.synchronize()
-    e0.record()
-    g.replay()
-    e1.record()
-    e1.synchronize()
-    graph_us = e0.elapsed_time(e1) * 1e3 / steps
+    def one_step(t):
+        a = per["alpha"][t].squeeze(-1)
+        b = per["beta"][t].squeeze(-1)
+        sdm.step(per["q"][t], per["k"][t], per["v"][t], a, b, C1, C2, M, topk=cfg.k,
+                 W=cfg.W, R=cfg.R, o=o[t])
+
+    def timed(one):
+        for t in range(min(steps, 8)):
+            one(t)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for t in range(steps):
+            one(t)
+        e1.record()
+        e1.synchronize()
+        eager_us = e0.elapsed_time(e1) * 1e3 / steps
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for t in range(steps):
+                    one(t)
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        graph_us = e0.elapsed_time(e1) * 1e3 / steps
+        del g
+        return {"eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
+                "graph_token_heads_per_s": cfg.BH / (graph_us * 1e-6)}
+
+    res = {"sdm_step": timed(one_step), "sdm_forward_T1": timed(one_forward)}
     st, info = sdm.device_status(ws)
-    del g
-    return {"decode": "sdm_forward per step (T = 1), M carried", "workload": workload_desc(cfg),
-            "steps": steps, "heads": cfg.BH, "eager_us_per_step": eager_us,
-            "graph_us_per_step": graph_us,
-            "graph_token_heads_per_s": cfg.BH / (graph_us * 1e-6), "device_status": st}
+    return {"decode": "one call per step, M carried", "workload": workload_desc(cfg),
+            "steps": steps, "heads": cfg.BH, "kernels": res, "device_status": st}
 
 
 def main():

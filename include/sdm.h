@@ -141,6 +141,30 @@ SDM_API int sdm_recur(const void* v, const float* alpha, const float* beta, cons
               void* stream);
 
 /*
+ * The forward pass for short calls -- decoding one step (T = 1) or a few at a
+ * time with M carried from call to call -- fused into one kernel that needs no
+ * workspace ("Mecanismo Central" items 1-4; the inference use of the method
+ * in "Resultados").  One CTA per (b,h) head runs the call's T steps in order,
+ * each on chip: scoring on CUDA cores (float32 FMA), the exact per-half top-k,
+ * the same staircase merge and softmax weights as sdm_forward, the gated delta
+ * writes, then the reads.  Same inputs, outputs and layouts as sdm_forward; o
+ * is reduced in a fixed order (identical calls give identical bits).  Its
+ * float32 scores can round differently from sdm_forward's (tensor cores) in the
+ * last bits, so the two may choose differently at exact near-ties only.
+ *   idx_w, w_w, idx_r, w_r: optional (all four NULL, or all four given): the
+ *     selections of every step in rank order, as sdm_select writes them.
+ * Sizes this kernel serves: n_sub <= 1024, k <= 256, d_v <= 128, d_qk/2 a
+ * power-of-two multiple of 8 (bf16) or 4 (float32) up to 32 times that, and
+ * its shared memory (staircase tables grow with W and R) within 227 KB;
+ * others return SDM_ERR_UNSUPPORTED before anything is enqueued.  Longer
+ * sequences are better served by sdm_forward.  Asynchronous on `stream`.
+ */
+SDM_API int sdm_step(const void* q, const void* k, const void* v, const float* alpha,
+                     const float* beta, const void* C1, const void* C2, float* M_inout,
+                     float* o_out, int32_t* idx_w, float* w_w, int32_t* idx_r, float* w_r,
+                     const sdm_dims* dims, void* stream);
+
+/*
  * sdm_forward that also records caller-created CUDA events (cudaEvent_t) on
  * `stream` at the boundaries of its kernel phases, for timing: for time chunk c
  * (see sdm_query_plan) events[5c+0] before scoring, [5c+1] after scoring,
@@ -186,7 +210,9 @@ SDM_API int sdm_forward_noalloc(const void* q, const void* k, const void* v, con
  * values into out: [0] tensor-core scoring (1) or CUDA-core scoring (0),
  * [1] survivor capacity per half-row, [2] steps per plan block P,
  * [3] recurrence streams per head S, [4] steps per time chunk, [5] number of
- * chunks, [6] kernel launches per sdm_forward call, [7] slot buckets per head.
+ * chunks, [6] kernel launches per sdm_forward call, [7] slot buckets per head,
+ * [8] scoring mode: 0 CUDA cores, 1 tensor cores with the exact top-k taken in
+ * the same kernel, 2 tensor-core threshold filter then a separate exact top-k.
  * Returns SDM_OK or a dims error.
  */
 SDM_API int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n);

@@ -509,6 +509,259 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
   }
 }
 
+// ---- filter-only variant --------------------------------------------------
+// k_score_tc_filter: the same TMA -> tcgen05 pipeline with 128-row codebook
+// tiles (two 128-column TMEM buffers, 256 columns per CTA, so that two CTAs
+// share an SM), and an epilogue of kQF = 2 threads per token row that only
+// filters: every score at or above the row's threshold is appended, unsorted,
+// to the half-row's survivor list in global memory (capacity C).  A row whose
+// kept count falls outside [k, C], or whose scores do not spread, is queued
+// for the exact CUDA-core path; the exact sorted top-k of the kept scores is
+// taken afterwards by k_topk_surv.  This needs no shared memory for the
+// survivors, so it serves every k (the in-kernel selection above needs about
+// 6 * C bytes per token row).
+constexpr int kTileNF = 128;
+constexpr int kQF = 2;
+constexpr int kEpiThreadsF = kQF * kTileM;
+constexpr int kThreadsF = 64 + kEpiThreadsF;
+constexpr int kStagesF = 2;
+constexpr uint32_t kBTileBytesF = kTileNF * 128;  // one 64-column chunk of a codebook tile
+
+struct TcLayoutF {
+  uint32_t a, b, rows, bars, total;
+  int nkc;
+};
+
+__host__ __device__ inline TcLayoutF tc_layout_f(const Plan& p) {
+  TcLayoutF L;
+  L.nkc = p.dh / kKAtom;
+  uint32_t o = 0;
+  L.a = o; o += L.nkc * kATileBytes;
+  L.b = o; o += kStagesF * L.nkc * kBTileBytesF;
+  L.rows = o; o += (1 + 2 * kQF) * kTileM * 4;  // per-row count, partial stats
+  o = (o + 15) & ~15u;
+  L.bars = o; o += 16 * 8;
+  L.total = o + 1024;
+  return L;
+}
+
+__device__ __forceinline__ void epi_sync_f() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreadsF) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreadsF, 2)
+k_score_tc_filter(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                  const __grid_constant__ CUtensorMap mc1, const __grid_constant__ CUtensorMap mc2,
+                  TcArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
+  const Plan& p = a.p;
+  const TcLayoutF L = tc_layout_f(p);
+  unsigned char* sA = smem + L.a;
+  unsigned char* sB = smem + L.b;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* full = bars;        // [kStagesF] TMA -> MMA
+  uint64_t* empty = bars + 2;   // [kStagesF] MMA -> TMA
+  uint64_t* a_full = bars + 4;
+  uint64_t* tfull = bars + 5;   // [2] MMA -> epilogue
+  uint64_t* tempty = bars + 7;  // [2] epilogue -> MMA
+  uint64_t* drain = bars + 9;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  volatile int* epi_abort = reinterpret_cast<volatile int*>(bars + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, bh = blockIdx.y, side = blockIdx.z >> 1, half = blockIdx.z & 1;
+  const int h = bh % p.H;
+  const int ntiles = p.n / kTileNF;
+  const int nk = p.dh / 16;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], kEpiThreadsF);
+    }
+    mbar_init(a_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *epi_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                     su32(const_cast<uint32_t*>(tmem_slot)))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      const CUtensorMap* mx = side ? &mq : &mk;
+      const CUtensorMap* mc = half ? &mc2 : &mc1;
+      tma_prefetch(mx);
+      tma_prefetch(mc);
+      const int row0 = bh * p.T + a.t0 + tile * kTileM;
+      mbar_expect_tx(a_full, L.nkc * kATileBytes);
+      for (int kc = 0; kc < L.nkc; ++kc)
+        tma_load_2d(mx, a_full, sA + kc * kATileBytes, half * p.dh + kc * kKAtom, row0);
+      int issued = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+        mbar_expect_tx(&full[s], L.nkc * kBTileBytesF);
+        for (int kc = 0; kc < L.nkc; ++kc)
+          tma_load_2d(mc, &full[s], sB + (s * L.nkc + kc) * kBTileBytesF, kc * kKAtom,
+                      h * p.n + j * kTileNF);
+        ++issued;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        mbar_wait(a_full, 0, &never);
+        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+          mbar_wait(&full[j & 1], (j >> 1) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kTileM, kTileNF);
+      int issued = 0;
+      if (mbar_wait(a_full, 0, abort_flag)) {
+        for (int j = 0; j < ntiles; ++j) {
+          const int s = j & 1;
+          if (!mbar_wait(&full[s], (j >> 1) & 1, abort_flag)) break;
+          if (j >= 2 && !mbar_wait(&tempty[s], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t d = tmem + uint32_t(s * kTileNF);
+          for (int kk = 0; kk < nk; ++kk) {
+            const int kc = kk >> 2, w = kk & 3;
+            const uint64_t ad = sdesc(su32(sA + kc * kATileBytes + w * 32));
+            const uint64_t bd = sdesc(su32(sB + (s * L.nkc + kc) * kBTileBytesF + w * 32));
+            umma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          umma_commit(&tfull[s]);
+          ++issued;
+        }
+      }
+      if (*abort_flag && issued > 0) {
+        umma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never);
+      }
+    }
+  } else {
+    // ---------------- epilogue: kQF threads per token row (= TMEM lane)
+    const int q4 = warp & 3;
+    const int sub = (warp - 2) >> 2;  // which half of every tile's columns
+    const int row = q4 * 32 + lane;
+    const int tl = tile * kTileM + row;
+    const bool valid = tl < a.tlen;
+    const uint32_t tbase = tmem + (uint32_t(q4 * 32) << 16);
+    const int C = p.C;
+    constexpr int kCols = kTileNF / kQF;  // 64
+    int* rcnt = reinterpret_cast<int*>(smem + L.rows);       // [128] kept count
+    float* rst = reinterpret_cast<float*>(rcnt + kTileM);    // [2][kQF][128] sum, sq
+    const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
+    uint2* g = a.surv + hr * C;
+    float v[32];
+    if (sub == 0) rcnt[row] = 0;
+    // statistics of the first (up to) two tiles
+    const int nstat = ntiles < 2 ? ntiles : 2;
+    float sum = 0.f, sq = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nstat && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&tfull[j], 0, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < kCols / 32; ++c) {
+        tmem_ld32(tbase + uint32_t(j * kTileNF + sub * kCols + c * 32), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sum += v[i];
+          sq = fmaf(v[i], v[i], sq);
+        }
+      }
+    }
+    if (!ok) *epi_abort = 1;
+    rst[(0 * kQF + sub) * kTileM + row] = sum;
+    rst[(1 * kQF + sub) * kTileM + row] = sq;
+    epi_sync_f();
+    ok = !*epi_abort;
+    const bool keep_all = !(a.z > -1e30f);
+    float tau;
+    bool redo;
+    {
+      float S = 0.f, S2 = 0.f;
+#pragma unroll
+      for (int j = 0; j < kQF; ++j) {
+        S += rst[(0 * kQF + j) * kTileM + row];
+        S2 += rst[(1 * kQF + j) * kTileM + row];
+      }
+      const float m = float(nstat * kTileNF);
+      const float mu = S / m;
+      const float sd = sqrtf(fmaxf(S2 / m - mu * mu, 0.f));
+      tau = keep_all ? -INFINITY : mu + a.z * sd;
+      redo = !keep_all && !(sd > 0.f);
+      if (!valid) tau = INFINITY;  // rows past the chunk keep nothing
+    }
+    // filter: append the kept scores of this thread's columns to the row's
+    // survivor list in global memory
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int s = j & 1;
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[s], (j >> 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int c = 0; c < kCols / 32; ++c) {
+        tmem_ld32(tbase + uint32_t(s * kTileNF + sub * kCols + c * 32), v);
+        const int col0 = j * kTileNF + sub * kCols + c * 32;
+        uint32_t mask = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mask |= (v[i] >= tau ? 1u : 0u) << i;
+        if (mask) {
+          int pos = atomicAdd(&rcnt[row], __popc(mask));
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if ((mask >> i) & 1u) {
+              if (pos < C) g[pos] = make_uint2(__float_as_uint(v[i]), uint32_t(col0 + i));
+              ++pos;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[s]);
+    }
+    if (!ok) *epi_abort = 1;
+    epi_sync_f();
+    ok = !*epi_abort;
+    if (!ok && threadIdx.x == 64) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
+    if (sub == 0 && valid) {
+      const int cnt = rcnt[row];
+      if (ok && !redo && cnt >= p.k && cnt <= C) a.cnt[hr] = cnt;
+      else a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);  // exact CUDA-core path
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -547,29 +800,52 @@ double normal_upper_quantile(double f) {
 
 }  // namespace
 
-// Survivor capacity of a half-row: room for the expected kept count
-// (1.5 k + 16) plus a margin of 48.
-int score_tc_capacity(const sdm_dims* d) {
-  int c = (3 * d->k) / 2 + 16 + 48;
+// Survivor capacity of a half-row.  In-kernel selection: room for the expected
+// kept count (1.5 k + 16) plus a margin of 48.  Filter only: the expected kept
+// count is 1.7 k + 16 (its threshold comes from 256 scores, not 512) and the
+// list lives in global memory, so the margin is wider: 2 k + 80.
+int score_tc_capacity(const sdm_dims* d, int mode) {
+  int c = mode == 2 ? 2 * d->k + 80 : (3 * d->k) / 2 + 16 + 48;
   c = (c + 15) & ~15;
   return c < d->n_sub ? c : d->n_sub;
 }
 
-size_t score_tc_smem(const Plan& p) { return tc_layout(p).total; }
+static double kept_target(const Plan& p) {
+  return p.tc == 2 ? 1.7 * p.k + 16.0 : 1.5 * p.k + 16.0;
+}
 
-bool score_tc_supported(const sdm_dims* d) {
-  if (d->in_dtype != SDM_DTYPE_BF16) return false;
+size_t score_tc_smem(const Plan& p) {
+  return p.tc == 2 ? tc_layout_f(p).total : tc_layout(p).total;
+}
+
+#ifndef SDM_TC_MODE
+#define SDM_TC_MODE 0  // 0: chosen by shape; 1 or 2: that mode wherever it runs
+#endif
+
+// Which tensor-core scoring kernel serves d: 0 none (CUDA cores), 1 k_score_tc
+// (in-kernel exact selection), 2 k_score_tc_filter + k_topk_surv.  Mode 1 is
+// preferred where its per-row survivor lists fit shared memory.
+int score_tc_mode(const sdm_dims* d) {
+  if (d->in_dtype != SDM_DTYPE_BF16) return 0;
   const int dh = d->d_qk / 2;
-  if (dh % kKAtom != 0 || dh > 256) return false;
-  if (d->n_sub % kTileN != 0 || d->n_sub > 65535) return false;
-  if ((long long)d->B * d->H * d->T >= (1LL << 31)) return false;
-  if ((long long)d->H * d->n_sub >= (1LL << 31)) return false;
+  if (dh % kKAtom != 0 || dh > 256) return 0;
+  if (d->n_sub % kTileNF != 0 || d->n_sub > 65535) return 0;
+  if ((long long)d->B * d->H * d->T >= (1LL << 31)) return 0;
+  if ((long long)d->H * d->n_sub >= (1LL << 31)) return 0;
   Plan tmp;
   tmp.dh = dh;
-  tmp.C = score_tc_capacity(d);
+  tmp.C = score_tc_capacity(d, 1);
+  tmp.tc = 1;
   const TcLayout L = tc_layout(tmp);
   // per-row bucket counts and offsets are packed bytes: the capacity stays below 256
-  return tmp.C <= 255 && L.total <= 227 * 1024 && out_capacity(L) >= d->k + 16;
+  const bool m1 = d->n_sub % kTileN == 0 && tmp.C <= 255 && L.total <= 227 * 1024 &&
+                  out_capacity(L) >= d->k + 16;
+  tmp.tc = 2;
+  tmp.C = score_tc_capacity(d, 2);
+  const bool m2 = tc_layout_f(tmp).total <= 227 * 1024;
+  if (SDM_TC_MODE == 1) return m1 ? 1 : 0;
+  if (SDM_TC_MODE == 2) return m2 ? 2 : 0;
+  return m1 ? 1 : (m2 ? 2 : 0);
 }
 
 cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const void* C1,
@@ -577,27 +853,35 @@ cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const v
                             int* redo_rows, DevStatus* st, cudaStream_t s) {
   CUtensorMap mq, mk, mc1, mc2;
   if (!encode_fn()) return cudaErrorNotSupported;
+  const uint32_t box_n = p.tc == 2 ? kTileNF : kTileN;
   const uint64_t rows = uint64_t(p.BH) * p.T;
   if (!make_map(&mq, q, rows, p.dqk, kTileM) || !make_map(&mk, k, rows, p.dqk, kTileM) ||
-      !make_map(&mc1, C1, uint64_t(p.H) * p.n, p.dh, kTileN) ||
-      !make_map(&mc2, C2, uint64_t(p.H) * p.n, p.dh, kTileN))
+      !make_map(&mc1, C1, uint64_t(p.H) * p.n, p.dh, box_n) ||
+      !make_map(&mc2, C2, uint64_t(p.H) * p.n, p.dh, box_n))
     return cudaErrorInvalidValue;
   TcArgs a;
   a.p = p;
   a.t0 = t0;
   a.tlen = tlen;
-  const double f = (1.5 * p.k + 16.0) / double(p.n);
+  const double f = kept_target(p) / double(p.n);
   a.z = (f >= 1.0 || p.C >= p.n) ? -INFINITY : float(normal_upper_quantile(f));
   a.surv = surv;
   a.cnt = surv_cnt;
   a.redo = redo_rows;
   a.st = st;
   const size_t smem = score_tc_smem(p);
-  cudaError_t e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
-  if (e != cudaSuccess) return e;
   dim3 grid((tlen + kTileM - 1) / kTileM, p.BH, 4);
-  k_score_tc<<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+  cudaError_t e;
+  if (p.tc == 2) {
+    e = cudaFuncSetAttribute(k_score_tc_filter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    k_score_tc_filter<<<grid, kThreadsF, smem, s>>>(mq, mk, mc1, mc2, a);
+  } else {
+    e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    k_score_tc<<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+  }
   return cudaGetLastError();
 }
 

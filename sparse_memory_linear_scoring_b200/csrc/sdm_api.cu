@@ -22,8 +22,6 @@ size_t score_simt_smem(const Plan& p);
 size_t merge_smem_bytes(const Plan& p, int warps);
 size_t plan_smem_bytes(const Plan& p);
 int recur_lanes_per_row(int dv);
-size_t score_tc_smem(const Plan& p);
-int score_tc_capacity(const sdm_dims* d);
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
@@ -67,9 +65,10 @@ int make_plan(const sdm_dims* d, Plan* p, size_t chunk_budget) {
   p->dtype = d->in_dtype;
   p->BH = d->B * d->H;
   p->N = (long long)d->n_sub * d->n_sub;
-  p->tc = score_tc_supported(d) ? 1 : 0;
+  p->tc = score_tc_mode(d);
+  if (p->tc == 2 && !topk_surv_supported(score_tc_capacity(d, 2))) p->tc = 0;
   if (!p->tc && d->n_sub > 4096) return SDM_ERR_UNSUPPORTED;
-  p->C = p->tc ? score_tc_capacity(d) : d->k;
+  p->C = p->tc ? score_tc_capacity(d, p->tc) : d->k;
   staircase(p->k, p->W, &p->ncW, &p->nfW);
   staircase(p->k, p->R, &p->ncR, &p->nfR);
   if (p->ncW < p->W || p->ncR < p->R) return SDM_ERR_UNSUPPORTED;
@@ -115,7 +114,7 @@ int make_plan(const sdm_dims* d, Plan* p, size_t chunk_budget) {
   p->recur_smem = 0;
   p->score_smem = p->tc ? score_tc_smem(*p) : score_simt_smem(*p);
   if (p->merge_smem > kMaxSmem || p->plan_smem > kMaxSmem || p->recur_smem > kMaxSmem ||
-      p->score_smem > kMaxSmem)
+      p->score_smem > kMaxSmem || (p->tc == 2 && topk_surv_smem(*p) > kMaxSmem))
     return SDM_ERR_UNSUPPORTED;
   const size_t nhr = size_t(p->BH) * p->Tc * 4;
   size_t o = 0;
@@ -207,7 +206,11 @@ static cudaError_t score_chunk(const Plan& p, const Carve& c, const void* q, con
     if ((e = launch_score_tc(p, q, k, C1, C2, t0, tlen, c.cnt, c.surv, c.redo, c.st, s)) !=
         cudaSuccess)
       return e;
-    return launch_score_simt(p, q, k, C1, C2, t0, tlen, c.redo, c.st, c.cnt, c.surv, c.st, s);
+    if ((e = launch_score_simt(p, q, k, C1, C2, t0, tlen, c.redo, c.st, c.cnt, c.surv, c.st,
+                               s)) != cudaSuccess)
+      return e;
+    // filter mode: the survivor lists are unsorted supersets; keep their exact top-k
+    return p.tc == 2 ? launch_topk_surv(p, tlen, c.cnt, c.surv, c.st, s) : cudaSuccess;
   }
   return launch_score_simt(p, q, k, C1, C2, t0, tlen, nullptr, nullptr, c.cnt, c.surv, c.st, s);
 }
@@ -298,10 +301,10 @@ extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
   Plan p;
   const int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
-  const int64_t per_chunk = (p.tc ? 3 : 1) + 2 + (p.BH + p.HG - 1) / p.HG;
+  const int64_t per_chunk = (p.tc == 2 ? 4 : p.tc ? 3 : 1) + 2 + (p.BH + p.HG - 1) / p.HG;
   const int64_t launches = 1 + per_chunk * p.nchunks - (p.tc && p.nchunks > 0 ? 1 : 0);
-  const int64_t vals[8] = {p.tc, p.C, p.P, p.S, p.Tc, p.nchunks, launches, p.NB};
-  for (int i = 0; i < n && i < 8; ++i) out[i] = vals[i];
+  const int64_t vals[9] = {p.tc ? 1 : 0, p.C, p.P, p.S, p.Tc, p.nchunks, launches, p.NB, p.tc};
+  for (int i = 0; i < n && i < 9; ++i) out[i] = vals[i];
   return SDM_OK;
 }
 

@@ -56,7 +56,8 @@ struct Plan {
   int B, H, T, dqk, dh, dv, n, k, W, R, dtype;
   int BH;
   long long N;
-  int tc;      // 1: tensor-core scoring, 0: SIMT scoring
+  int tc;      // scoring mode: 0 CUDA cores, 1 tensor cores + in-kernel selection,
+               // 2 tensor-core filter + survivor top-k (score_tc_mode)
   int C;       // survivor capacity per half-row
   int Tc;      // steps per chunk
   int nchunks;
@@ -150,7 +151,7 @@ __device__ __forceinline__ void warp_sort_desc(uint64_t* a, int S) {
   }
 }
 
-inline int next_pow2(int x) {
+__host__ __device__ inline int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;
   return p;
@@ -165,7 +166,17 @@ cudaError_t launch_score_simt(const Plan& p, const void* q, const void* k, const
 cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const void* C1,
                             const void* C2, int t0, int tlen, int* surv_cnt, uint2* surv,
                             int* redo_rows, DevStatus* st, cudaStream_t s);
-bool score_tc_supported(const sdm_dims* d);
+// 0: CUDA-core scoring; 1: k_score_tc (in-kernel exact selection); 2:
+// k_score_tc_filter (unsorted survivor lists), then k_topk_surv.
+int score_tc_mode(const sdm_dims* d);
+int score_tc_capacity(const sdm_dims* d, int mode);
+size_t score_tc_smem(const Plan& p);
+bool topk_surv_supported(int C);
+size_t topk_surv_smem(const Plan& p);
+// In place: the exact sorted top-k of every half-row's survivor list of the
+// chunk's first tlen steps (counts become k).
+cudaError_t launch_topk_surv(const Plan& p, int tlen, int* cnt, uint2* surv, DevStatus* st,
+                             cudaStream_t s);
 
 // Lists of (slot, weight) pairs: iw/ww [rows][W], ir/wr [rows][R]; a step's
 // row is bh * list_T + list_t0 + (step within the chunk).

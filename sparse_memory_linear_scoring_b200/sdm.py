@@ -62,6 +62,8 @@ def load_library():
             lib.sdm_forward_timed.restype = ctypes.c_int
             lib.sdm_query_plan.argtypes = [DP, P, ctypes.c_int]
             lib.sdm_query_plan.restype = ctypes.c_int
+            lib.sdm_step.argtypes = [P] * 13 + [DP, P]
+            lib.sdm_step.restype = ctypes.c_int
             lib.sdm_version.argtypes = []
             lib.sdm_version.restype = ctypes.c_int
             _lib = lib
@@ -190,7 +192,7 @@ def _stream(dev, stream):
 
 
 PLAN_FIELDS = ("tensor_core_scoring", "survivor_capacity", "block_steps", "streams_per_head",
-               "chunk_steps", "chunks", "launches_per_call", "buckets_per_head")
+               "chunk_steps", "chunks", "launches_per_call", "buckets_per_head", "scoring_mode")
 
 
 def query_plan(dims: Dims) -> Dict[str, int]:
@@ -231,6 +233,35 @@ def forward(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
                            _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws), _nbytes(ws),
                            _stream(dev, stream)))
     return o
+
+
+def step(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
+         o: Optional[torch.Tensor] = None, lists: bool = False, stream=None):
+    """Short calls (decoding) through the fused single-step kernel (sdm_step):
+    same arguments and layouts as forward (T steps, typically 1), no workspace.
+    Returns o, or (o, idx_w, w_w, idx_r, w_r) with lists=True."""
+    B, H, T, d_qk, n_sub, dt = _check_inputs(q, k, v, C1, C2, alpha, beta)
+    d_v = v.shape[-1]
+    _expect(M, "M", (B, H, n_sub * n_sub, d_v), (torch.float32,))
+    if o is not None:
+        _expect(o, "o", (B, H, T, d_v), (torch.float32,))
+    dev = _dev(q, k, v, alpha, beta, C1, C2, M, *([o] if o is not None else []))
+    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, W, R, dt)
+    if o is None:
+        o = torch.empty(B, H, T, d_v, dtype=torch.float32, device=dev)
+    outs = [("M", M), ("o", o)]
+    lw = [None] * 4
+    if lists:
+        lw = [torch.empty(B, H, T, W, dtype=torch.int32, device=dev),
+              torch.empty(B, H, T, W, dtype=torch.float32, device=dev),
+              torch.empty(B, H, T, R, dtype=torch.int32, device=dev),
+              torch.empty(B, H, T, R, dtype=torch.float32, device=dev)]
+    _no_alias(outs, [("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                     ("C1", C1), ("C2", C2)])
+    _check(load_library().sdm_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(C1),
+                                   _ptr(C2), _ptr(M), _ptr(o), *[_ptr(x) for x in lw],
+                                   ctypes.byref(dims), _stream(dev, stream)))
+    return (o, *lw) if lists else o
 
 
 def select(q, k, C1, C2, *, topk: int, W: int, R: int, d_v: int = 4,

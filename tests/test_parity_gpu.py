@@ -133,10 +133,31 @@ def test_tensor_core_scoring_shapes(shape):
     _check_forward(cfg, inp, ref)
 
 
+@pytest.mark.parametrize("shape", [
+    dict(), dict(T=1), dict(T=129), dict(T=300, B=2, H=1),
+    dict(d_qk=128, d_v=64, n_sub=512, k=128, W=128, R=128, T=200),
+    dict(d_qk=128, d_v=64, n_sub=384, k=32, W=64, R=64, T=200),
+    dict(d_qk=128, d_v=64, n_sub=128, k=16, W=32, R=32, T=200),
+    dict(d_qk=256, d_v=32, n_sub=256, k=64, W=100, R=37, T=150),
+])
+def test_tensor_core_filter_shapes(shape):
+    """bf16 shapes served by the tensor-core threshold filter and the survivor
+    top-k (scoring mode 2): the long-context shape (d_h = 128, k = W = R = 128,
+    recurring keys) with ragged and single steps, k = 128 at d_h = 64, and
+    codebooks of 128 and 384 rows."""
+    base = config(3).with_(B=1, H=2, T=300, m0_sd=0.5)
+    cfg = base.with_(**shape)
+    assert sdm.query_plan(sdm.make_dims(**cfg.dims()))["scoring_mode"] == 2
+    inp = gen_inputs(cfg)
+    ref = oracle_full(inp, cfg, lists=True)
+    _check_forward(cfg, inp, ref)
+
+
 @pytest.mark.parametrize("base", [
     config(1).with_(B=1, H=2, T=200, n_sub=256, k=32, W=64, R=64, m0_sd=0.5),
+    config(3).with_(B=1, H=2, T=120, m0_sd=0.5),
     config(0).with_(B=1, H=2, T=150, m0_sd=0.5),
-], ids=["bf16-tensor-core", "fp32"])
+], ids=["bf16-tensor-core", "bf16-tensor-core-filter", "fp32"])
 def test_duplicate_codebook_rows(base):
     """Duplicated codebook rows make exact score ties at every rank: the lower
     index must win in each half and among slots, on the GPU as in the oracle."""
@@ -231,10 +252,15 @@ def test_repeated_slots(period, share):
     _check_forward(cfg, inp, ref)
 
 
-def test_all_zero_keys_and_queries():
+@pytest.mark.parametrize("base", [
+    config(1).with_(B=1, H=2, T=200, n_sub=64, k=16, W=24, R=16, m0_sd=0.5),
+    config(3).with_(B=1, H=1, T=100, m0_sd=0.5),
+], ids=["cuda-cores", "tensor-core-filter"])
+def test_all_zero_keys_and_queries(base):
     """Every score is 0: every step selects the lowest slots (ties go to the
-    lower index), so each plan block holds the same few slots P times over."""
-    cfg = config(1).with_(B=1, H=2, T=200, n_sub=64, k=16, W=24, R=16, m0_sd=0.5)
+    lower index), so each plan block holds the same few slots P times over (on
+    the tensor-core filter path every row is re-scored exactly)."""
+    cfg = base
     inp = gen_inputs(cfg)
     inp["q"] = torch.zeros_like(inp["q"])
     inp["k"] = torch.zeros_like(inp["k"])
