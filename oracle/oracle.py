@@ -17,6 +17,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 ORACLE_SRC = os.path.join(_HERE, "sdm_oracle.c")
 ORACLE_SO = os.path.join(_HERE, "libsdm_oracle.so")
+GDN_SRC = os.path.join(_HERE, "gdn_oracle.c")
+GDN_SO = os.path.join(_HERE, "libgdn_oracle.so")
 
 _libs = {}
 _lock = threading.Lock()
@@ -33,11 +35,13 @@ def compile_source(src: str, so: str) -> str:
 
 
 def build(force: bool = False) -> str:
-    """Compile oracle/sdm_oracle.c into oracle/libsdm_oracle.so (if stale)."""
-    if (not force and os.path.exists(ORACLE_SO)
-            and os.path.getmtime(ORACLE_SO) >= os.path.getmtime(ORACLE_SRC)):
-        return ORACLE_SO
-    return compile_source(ORACLE_SRC, ORACLE_SO)
+    """Compile oracle/sdm_oracle.c into oracle/libsdm_oracle.so and
+    oracle/gdn_oracle.c into oracle/libgdn_oracle.so (each if stale)."""
+    for src, so in ((GDN_SRC, GDN_SO), (ORACLE_SRC, ORACLE_SO)):
+        if (force or not os.path.exists(so)
+                or os.path.getmtime(so) < os.path.getmtime(src)):
+            compile_source(src, so)
+    return ORACLE_SO
 
 
 def load(so: Optional[str] = None):
@@ -155,3 +159,45 @@ def select(x, C1, C2, dims: Dict[str, int], n_sel: int, so: Optional[str] = None
     if rc != 0:
         raise ValueError("oracle rejected the dimensions")
     return slots, w, s, flag.value
+
+
+# ---------------------------------------------------------------- dense GDN
+def load_gdn(so: Optional[str] = None):
+    """ctypes handle of the GDN oracle (the default build, or another .so)."""
+    with _lock:
+        if so is None:
+            so = GDN_SO
+            if (not os.path.exists(so)) or os.path.getmtime(so) < os.path.getmtime(GDN_SRC):
+                compile_source(GDN_SRC, so)
+        if so not in _libs:
+            lib = ctypes.CDLL(so)
+            P = ctypes.c_void_p
+            lib.gdn_oracle_forward.argtypes = [P] * 7 + [P, ctypes.c_int, ctypes.c_int,
+                                                         ctypes.c_int]
+            lib.gdn_oracle_forward.restype = ctypes.c_int
+            _libs[so] = lib
+        return _libs[so]
+
+
+def gdn_forward(inp: Dict[str, np.ndarray], dims: Dict[str, int], t_begin: int = 0,
+                t_end: Optional[int] = None, nthreads: int = 1, S=None,
+                so: Optional[str] = None) -> Dict[str, np.ndarray]:
+    """The dense GDN oracle (gdn_oracle_forward).  inp: q, k [B,H,T,d_k];
+    v [B,H,T,d_v]; alpha, beta [B,H,T]; S0 [B,H,d_v,d_k] (ignored when S is
+    given; S is then updated in place).  dims: B, H, T, d_k, d_v.
+    Returns o [B,H,T,d_v] and S."""
+    lib = load_gdn(so)
+    T = dims['T']
+    t_end = T if t_end is None else t_end
+    q, k, v = _f32(inp['q']), _f32(inp['k']), _f32(inp['v'])
+    al, be = _f32(inp['alpha']), _f32(inp['beta'])
+    if S is None:
+        S = _f32(inp['S0']).copy()
+    assert S.dtype == np.float32 and S.flags['C_CONTIGUOUS']
+    o = np.zeros((dims['B'], dims['H'], T, dims['d_v']), dtype=np.float32)
+    d = np.array([dims['B'], dims['H'], T, dims['d_k'], dims['d_v']], dtype=np.int32)
+    rc = lib.gdn_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(al), _ptr(be), _ptr(S), _ptr(o),
+                                _ptr(d), int(t_begin), int(t_end), int(nthreads))
+    if rc != 0:
+        raise ValueError("GDN oracle rejected the dimensions or ran out of memory")
+    return {'o': o, 'S': S}

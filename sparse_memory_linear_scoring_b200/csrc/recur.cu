@@ -170,16 +170,23 @@ __device__ __forceinline__ void cp_bytes(void* dst, const void* src) {
   }
 }
 
+#ifndef SDM_RECUR_VREG
+#define SDM_RECUR_VREG 0
+#endif
+
 template <typename Tv, int LPR, int F>
 struct RecurSmem {
   static constexpr int dv = LPR * F;
   static constexpr int U = kRecurChunk;
   static constexpr int kStreams = kRecurThreads / LPR;
+  // bf16 v rows are held in registers (F / 2 words a record), float32 ones
+  // are staged in shared memory
+  static constexpr bool kVReg = SDM_RECUR_VREG && sizeof(Tv) == 2;
   // per stream: two chunks of records (the one applied, the one arriving),
-  // then the chunk's rows of M and of v
+  // then the chunk's rows of M (and of v)
   static constexpr size_t ring = size_t(2) * U * 16;
   static constexpr size_t mrow = size_t(U) * dv * 4;
-  static constexpr size_t vrow = (size_t(U) * dv * sizeof(Tv) + 15) & ~size_t(15);
+  static constexpr size_t vrow = kVReg ? 0 : (size_t(U) * dv * sizeof(Tv) + 15) & ~size_t(15);
   static constexpr size_t per_stream = ring + mrow + vrow;
   static constexpr size_t total = per_stream * kStreams;
 };
@@ -309,9 +316,11 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
       pre_b = -1;
     }
     // gather into shared memory: the first record of every slot run copies
-    // the row; writes copy v_t.  Each lane copies and later reads only its own
-    // F columns, so its own wait makes them visible.
+    // the row; writes copy v_t (or load it into registers).  Each lane copies
+    // and later reads only its own F columns, so its own wait makes them
+    // visible.
     uint32_t head = 0, last = 0;  // per record: first / last of its slot run
+    VRaw<Tv, F> vr[SM::kVReg ? U : 1];
     {
       int prev = -1;
 #pragma unroll
@@ -324,7 +333,9 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
           cp_bytes<F * 4>(mrow + u * dv, Mh + size_t(unsigned(sm.x)) * dv);
         }
         if (!(sm.y & 1)) {
-          if constexpr (F * sizeof(Tv) >= 4)
+          if constexpr (SM::kVReg)
+            ld_v<Tv, F>(vh + size_t(sm.y >> 1) * dv, vr[SM::kVReg ? u : 0]);
+          else if constexpr (F * sizeof(Tv) >= 4)
             cp_bytes<F * sizeof(Tv)>(vrow + u * dv, vh + size_t(sm.y >> 1) * dv);
           else
             vrow[u * dv] = vh[size_t(sm.y >> 1) * dv];
@@ -350,7 +361,12 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
         }
         if (!(r.y & 1)) {
 #pragma unroll
-          for (int j = 0; j < F; ++j) cur[j] = fmaf(f1, cur[j], f2 * to_f32(vrow[u * dv + j]));
+          for (int j = 0; j < F; ++j) {
+            float vj;
+            if constexpr (SM::kVReg) vj = v_at<Tv, F>(vr[SM::kVReg ? u : 0], j);
+            else vj = to_f32(vrow[u * dv + j]);
+            cur[j] = fmaf(f1, cur[j], f2 * vj);
+          }
           dirty = true;
         } else {
           red_row<F>(oh + size_t(r.y >> 1) * dv, cur, f1);

@@ -1,0 +1,74 @@
+"""The dense GDN oracle against its pins (tests/gdn_pins.py), and plausible
+mistakes planted in copies of it (on the CPU) that each pin set must catch."""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+import gdn_pins
+import oracle
+
+
+@pytest.mark.parametrize("pin", gdn_pins.GDN_PINS, ids=lambda f: f.__name__)
+def test_gdn_oracle_pin(pin):
+    pin(None)
+
+
+GDN_MUTANTS = {
+    "prediction-from-ungated-state": lambda s: s.replace(
+        "        s[j] = a * s[j];\n        pred += s[j] * (double)kt[j];",
+        "        pred += s[j] * (double)kt[j];\n        s[j] = a * s[j];"),
+    "forget-gate-dropped": lambda s: s.replace("        s[j] = a * s[j];\n", ""),
+    "delta-sign-flipped": lambda s: s.replace(
+        "for (int j = 0; j < dk; ++j) s[j] += e * (double)kt[j];",
+        "for (int j = 0; j < dk; ++j) s[j] -= e * (double)kt[j];"),
+    "beta-dropped": lambda s: s.replace(
+        "const double e = b * ((double)vt[i] - pred);", "const double e = ((double)vt[i] - pred);"),
+    "update-along-query": lambda s: s.replace(
+        "for (int j = 0; j < dk; ++j) s[j] += e * (double)kt[j];",
+        "for (int j = 0; j < dk; ++j) s[j] += e * (double)qt[j];"),
+    "read-with-key": lambda s: s.replace(
+        "for (int j = 0; j < dk; ++j) o += s[j] * (double)qt[j];",
+        "for (int j = 0; j < dk; ++j) o += s[j] * (double)kt[j];"),
+    "read-before-write": lambda s: s.replace(
+        "      double pred = 0.0;\n",
+        "      double o0 = 0.0;\n      for (int j = 0; j < dk; ++j) o0 += a * s[j] * (double)qt[j];\n"
+        "      double pred = 0.0;\n").replace(
+        "      if (J->o) J->o[(tq + t) * dv + i] = (float)o;",
+        "      (void)o;\n      if (J->o) J->o[(tq + t) * dv + i] = (float)o0;"),
+}
+
+
+@pytest.fixture(scope="module")
+def mutant_dir():
+    with tempfile.TemporaryDirectory(prefix="gdn_oracle_mut_") as d:
+        yield d
+
+
+@pytest.mark.parametrize("name", sorted(GDN_MUTANTS))
+def test_gdn_mutant_is_caught(name, mutant_dir):
+    with open(oracle.GDN_SRC) as f:
+        src = f.read()
+    bad = GDN_MUTANTS[name](src)
+    assert bad != src, "mutation %s did not apply" % name
+    c = os.path.join(mutant_dir, name + ".c")
+    so = os.path.join(mutant_dir, name + ".so")
+    with open(c, "w") as f:
+        f.write(bad)
+    oracle.compile_source(c, so)
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import gdn_pins\n"
+            "bad = []\n"
+            "for pin in gdn_pins.GDN_PINS:\n"
+            "    try:\n"
+            "        pin(%r)\n"
+            "    except AssertionError:\n"
+            "        bad.append(pin.__name__)\n"
+            "print(bad)\n"
+            "sys.exit(1 if bad else 0)\n") % (here, os.path.dirname(here), so)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, "no pin catches the mutation %r" % name
+    assert r.stdout.strip() not in ("", "[]"), r.stderr
