@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--decode", action="store_true",
                     help="time single-step calls (T = 1, M carried), eagerly and as one CUDA "
                          "graph of --steps steps, on the workload's heads, and exit")
+    ap.add_argument("--gdn", action="store_true",
+                    help="time the dense Gated DeltaNet baseline at the matched size (d_k = W, "
+                         "same B, H, T, d_v, gates) beside the SDM forward pass, and exit")
     ap.add_argument("--probe-rows", action="store_true",
                     help="measure the HBM ceiling of random 256-byte row gathers and "
                          "read-modify-writes (the recurrence's access pattern) and exit")
@@ -637,6 +640,58 @@ def decode(cfg, steps):
             "steps": steps, "heads": cfg.BH, "kernels": res, "device_status": st}
 
 
+def gdn_compare(cfg, steps, warmup):
+    """The pages compare SDM with a dense Gated DeltaNet at matched FLOPs
+    (W = R = the GDN query dimension): time sdm_gdn_forward at d_k = W with the
+    workload's B, H, T, d_v and gates, and sdm_forward on the workload itself,
+    in the same process (CUDA events, L2 flushed before each step)."""
+    import torch
+    import sparse_memory_linear_scoring_b200 as sdm
+    from synth import gen_gdn_inputs, gen_inputs
+    dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
+    g = gen_gdn_inputs(cfg, device="cuda")
+    g = {n: (v.to(dt) if n in ("q", "k", "v") else v).contiguous() for n, v in g.items()}
+    ws = torch.empty(sdm.gdn_workspace_bytes(cfg.B, cfg.H, cfg.T, cfg.W, cfg.d_v, dt),
+                     dtype=torch.uint8, device="cuda")
+    og = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device="cuda")
+    S = g["S0"].clone()
+    d = gen_inputs(cfg, device="cuda")
+    d = {n: (v.to(dt) if n in ("q", "k", "v", "C1", "C2") else v).contiguous()
+         for n, v in d.items()}
+    M = d["M0"]
+    osd = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d_v, dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def time_it(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / steps
+
+    gdn_ms = time_it(lambda: sdm.gdn_forward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], S,
+                                             o=og, workspace=ws))
+    sdm_ms = time_it(lambda: sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"],
+                                         d["C2"], M, topk=cfg.k, W=cfg.W, R=cfg.R, o=osd))
+    th = cfg.BH * cfg.T
+    return {"baseline": "dense Gated DeltaNet (sdm_gdn_forward), matched d_k = W",
+            "workload": workload_desc(cfg), "gdn": {"d_k": cfg.W, "d_v": cfg.d_v,
+                                                    "ms_per_step": gdn_ms,
+                                                    "token_heads_per_s": th / (gdn_ms / 1e3)},
+            "sdm": {"ms_per_step": sdm_ms, "token_heads_per_s": th / (sdm_ms / 1e3)},
+            "sdm_over_gdn_time": sdm_ms / gdn_ms,
+            "pages": "SDM trains 1.49x slower than GDN at 8B (other hardware, training)",
+            "steps": steps, "l2": "flushed before each step"}
+
+
 def main():
     args = parse()
     if args.decode:
@@ -645,6 +700,11 @@ def main():
         return 0
     if args.probe_rows:
         print(json.dumps(probe_rows()), flush=True)
+        return 0
+    if args.gdn:
+        from synth import config as _config
+        print(json.dumps(gdn_compare(_config(args.config), max(3, min(args.steps, 200)),
+                                     max(3, args.warmup))), flush=True)
         return 0
     from synth import config
     cfg = config(args.config)

@@ -229,6 +229,39 @@ SDM_API int sdm_get_device_status(const void* workspace, size_t ws_bytes, int32_
 /* Static text for a return code (never NULL). */
 SDM_API const char* sdm_status_string(int status);
 
+/*
+ * Dense Gated DeltaNet (GDN) baseline, for comparison at matched sizes (the
+ * SDM summaries' "Resultados": SDM trains 1.49x slower than the dense GDN, an
+ * HBM-against-SRAM difference).  Per (b,h) head a dense state S in
+ * R^{d_v x d_k} follows the gated delta rule in the SDM pages' gate order
+ * ("Mecanismo Central" item 3 applied densely; the delta-mem page's section
+ * 2.A writes the dense rule):
+ *     S~ = alpha_t S_{t-1};  S_t = S~ + beta_t (v_t - S~ k_t) k_t^T;  o_t = S_t q_t.
+ * Evaluated in chunks of 64 steps in float32 on CUDA cores: a parallel pass
+ * over all (head, chunk) pairs solves each chunk's unit-lower-triangular
+ * system, then a pass per head and block of 8 rows of S walks the chunks in
+ * order.  Layouts: q, k [B][H][T][d_k] and v [B][H][T][d_v] (in_dtype);
+ * alpha, beta [B][H][T] float32 (alpha > 0); S_inout [B][H][d_v][d_k] float32,
+ * read as S_0 and overwritten with S_T; o_out [B][H][T][d_v] float32.  d_k, d_v
+ * in {16, 32, 64, 128}.  Keys are expected L2-normalised, as GDN uses them
+ * (the delta-mem page normalises q and k for stability).  The workspace holds
+ * the per-chunk quantities (sdm_gdn_workspace_bytes, which grows with T).
+ * Same pointer, stream and error conventions as sdm_forward.
+ */
+typedef struct sdm_gdn_dims {
+  int32_t B, H, T;
+  int32_t d_k;      /* key / query width */
+  int32_t d_v;      /* value width (rows of S) */
+  int32_t in_dtype; /* SDM_DTYPE_F32 or SDM_DTYPE_BF16, for q, k, v */
+} sdm_gdn_dims;
+
+SDM_API size_t sdm_gdn_workspace_bytes(const sdm_gdn_dims* dims);
+
+SDM_API int sdm_gdn_forward(const void* q, const void* k, const void* v, const float* alpha,
+                            const float* beta, float* S_inout, float* o_out,
+                            const sdm_gdn_dims* dims, void* workspace, size_t ws_bytes,
+                            void* stream);
+
 /* Library version, major*10000 + minor*100 + patch. */
 SDM_API int sdm_version(void);
 

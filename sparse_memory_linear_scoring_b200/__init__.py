@@ -8,5 +8,5 @@ without the built library, or with CPU tensors, raises.
 """
 from .sdm import (  # noqa: F401
     SDMError, Dims, LIB_PATH, load_library, workspace_bytes, forward, step, select, recur,
-    device_status, make_dims, query_plan, PLAN_FIELDS,
+    device_status, make_dims, query_plan, PLAN_FIELDS, gdn_forward, gdn_workspace_bytes, GdnDims,
 )

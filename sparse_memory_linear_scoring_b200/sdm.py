@@ -29,6 +29,10 @@ class Dims(ctypes.Structure):
         return {n: int(getattr(self, n)) for n, _ in self._fields_}
 
 
+class GdnDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "d_k", "d_v", "in_dtype")]
+
+
 _lib = None
 _lock = threading.Lock()
 _ws_cache: Dict[Tuple[int, int], torch.Tensor] = {}
@@ -62,6 +66,10 @@ def load_library():
             lib.sdm_forward_timed.restype = ctypes.c_int
             lib.sdm_query_plan.argtypes = [DP, P, ctypes.c_int]
             lib.sdm_query_plan.restype = ctypes.c_int
+            lib.sdm_gdn_workspace_bytes.argtypes = [ctypes.POINTER(GdnDims)]
+            lib.sdm_gdn_workspace_bytes.restype = S
+            lib.sdm_gdn_forward.argtypes = [P] * 7 + [ctypes.POINTER(GdnDims), P, S, P]
+            lib.sdm_gdn_forward.restype = ctypes.c_int
             lib.sdm_step.argtypes = [P] * 13 + [DP, P]
             lib.sdm_step.restype = ctypes.c_int
             lib.sdm_version.argtypes = []
@@ -262,6 +270,50 @@ def step(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
                                    _ptr(C2), _ptr(M), _ptr(o), *[_ptr(x) for x in lw],
                                    ctypes.byref(dims), _stream(dev, stream)))
     return (o, *lw) if lists else o
+
+
+def gdn_forward(q, k, v, alpha, beta, S, *, o: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense Gated DeltaNet baseline (sdm_gdn_forward).  q, k [B,H,T,d_k];
+    v [B,H,T,d_v] (one dtype, float32 or bfloat16); alpha, beta [B,H,T] float32;
+    S [B,H,d_v,d_k] float32, updated in place to S_T.  Returns o [B,H,T,d_v]."""
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q must be [B, H, T, d_k] and v [B, H, T, d_v]")
+    B, H, T, d_k = q.shape
+    d_v = v.shape[-1]
+    if q.dtype not in _IN_DTYPES:
+        raise TypeError("q has dtype %s, expected torch.float32 or torch.bfloat16" % q.dtype)
+    _expect(k, "k", (B, H, T, d_k), (q.dtype,))
+    _expect(v, "v", (B, H, T, d_v), (q.dtype,))
+    _expect(alpha, "alpha", (B, H, T), (torch.float32,))
+    _expect(beta, "beta", (B, H, T), (torch.float32,))
+    _expect(S, "S", (B, H, d_v, d_k), (torch.float32,))
+    if o is not None:
+        _expect(o, "o", (B, H, T, d_v), (torch.float32,))
+    dev = _dev(q, k, v, alpha, beta, S, *([o] if o is not None else []))
+    dims = GdnDims(int(B), int(H), int(T), int(d_k), int(d_v), _IN_DTYPES[q.dtype])
+    if o is None:
+        o = torch.empty(B, H, T, d_v, dtype=torch.float32, device=dev)
+    _no_alias([("S", S), ("o", o)], [("q", q), ("k", k), ("v", v), ("alpha", alpha),
+                                     ("beta", beta)])
+    lib = load_library()
+    need = int(lib.sdm_gdn_workspace_bytes(ctypes.byref(dims)))
+    if need == 0:
+        _check(lib.sdm_gdn_forward(*([None] * 7), ctypes.byref(dims), None, 0, None))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or _nbytes(workspace) < need or not workspace.is_contiguous():
+        raise SDMError(4, "workspace too small, not contiguous or on another device")
+    _check(lib.sdm_gdn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                               _ptr(o), ctypes.byref(dims), _ptr(workspace), _nbytes(workspace),
+                               _stream(dev, stream)))
+    return o
+
+
+def gdn_workspace_bytes(B, H, T, d_k, d_v, in_dtype) -> int:
+    dt = _IN_DTYPES[in_dtype] if isinstance(in_dtype, torch.dtype) else int(in_dtype)
+    dims = GdnDims(int(B), int(H), int(T), int(d_k), int(d_v), dt)
+    return int(load_library().sdm_gdn_workspace_bytes(ctypes.byref(dims)))
 
 
 def select(q, k, C1, C2, *, topk: int, W: int, R: int, d_v: int = 4,

@@ -48,6 +48,7 @@ _MIX2_S = _s64(_MIX2)
 # tensor ids of the streams
 TID_Q, TID_K, TID_V, TID_ALPHA, TID_BETA, TID_C1, TID_C2, TID_M0 = 1, 2, 3, 4, 5, 6, 7, 8
 TID_PATTERN, TID_PICK, TID_NOISE = 9, 10, 11
+TID_GDN_Q, TID_GDN_K, TID_GDN_S0 = 12, 13, 14
 
 
 def _mix_int(z: int) -> int:
@@ -246,4 +247,33 @@ def _gen(cfg, bs, hs, seed, device, t_end, with_m0, squeeze):
                 out[name] = out[name][0]
             else:
                 out[name] = out[name][0, 0]
+    return out
+
+
+def gen_gdn_inputs(cfg: SDMConfig, d_k: Optional[int] = None, seed: int = 0, device: str = 'cpu',
+                   s0_sd: float = 0.0, t_end: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Inputs of the dense Gated DeltaNet baseline matched to an SDM workload:
+    same B, H, T, d_v, gates and value stream; q', k' of width d_k (default W,
+    the matched query dimension) drawn N(0, I) and L2-normalised in float64
+    before rounding to the input dtype (GDN normalises its keys and queries);
+    S_0 = 0 unless s0_sd > 0.  Shapes: q, k [B,H,T,d_k], v [B,H,T,d_v],
+    alpha, beta [B,H,T], S0 [B,H,d_v,d_k] (float32 values)."""
+    d_k = cfg.W if d_k is None else d_k
+    T = cfg.T if t_end is None else t_end
+    bs, hs = list(range(cfg.B)), list(range(cfg.H))
+    out = {}
+    for name, tid in (('q', TID_GDN_Q), ('k', TID_GDN_K)):
+        x = _normals(cfg, seed, tid, bs, hs, (T, d_k), device)
+        out[name] = _round_input(x / torch.linalg.vector_norm(x, dim=-1, keepdim=True),
+                                 cfg.in_dtype)
+    out['v'] = _round_input(_normals(cfg, seed, TID_V, bs, hs, (T, cfg.d_v), device), cfg.in_dtype)
+    za = _normals(cfg, seed, TID_ALPHA, bs, hs, (T,), device)
+    zb = _normals(cfg, seed, TID_BETA, bs, hs, (T,), device)
+    out['alpha'] = torch.sigmoid(cfg.alpha_mu + cfg.alpha_sd * za).to(torch.float32)
+    out['beta'] = torch.sigmoid(cfg.beta_mu + cfg.beta_sd * zb).to(torch.float32)
+    if s0_sd > 0:
+        out['S0'] = (s0_sd * _normals(cfg, seed, TID_GDN_S0, bs, hs, (cfg.d_v, d_k),
+                                      device)).to(torch.float32)
+    else:
+        out['S0'] = torch.zeros(cfg.B, cfg.H, cfg.d_v, d_k, dtype=torch.float32, device=device)
     return out

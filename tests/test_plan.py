@@ -49,15 +49,18 @@ def test_plan_invariants(dims):
 @pytest.mark.parametrize("dims", SHAPES, ids=lambda d: "B%dH%dT%dn%d" % (d["B"], d["H"], d["T"], d["n_sub"]))
 def test_launch_count(dims):
     """Per chunk: scoring (tensor cores: filter + exact fallback, plus a reset of
-    the fallback list after the first chunk; else one kernel), merge, plan, and
-    one recurrence launch per head group; one status reset per call."""
+    the fallback list after the first chunk, plus the survivor top-k in the
+    filter-only mode; else one kernel), merge, plan, and one recurrence launch
+    per head group; one status reset per call."""
     plan = sdm.query_plan(sdm.make_dims(**dims))
     BH = dims["B"] * dims["H"]
     table = dims["n_sub"] ** 2 * dims["d_v"] * 4
     HG = max(1, min(BH, GROUP_BYTES // table))
     groups = -(-BH // HG)
     tc, nch = plan["tensor_core_scoring"], plan["chunks"]
-    per_chunk = (3 if tc else 1) + 2 + groups
+    mode = plan["scoring_mode"]
+    assert (mode > 0) == (tc == 1)
+    per_chunk = (4 if mode == 2 else 3 if tc else 1) + 2 + groups
     assert plan["launches_per_call"] == 1 + per_chunk * nch - (1 if tc and nch else 0)
 
 
