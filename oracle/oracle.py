@@ -59,6 +59,10 @@ def load(so: Optional[str] = None):
             lib.sdm_oracle_forward.restype = ctypes.c_int
             lib.sdm_oracle_select.argtypes = [P, P, P, P, ctypes.c_int, P, P, P, P]
             lib.sdm_oracle_select.restype = ctypes.c_int
+            if hasattr(lib, "sdm_oracle_forward_decay"):
+                lib.sdm_oracle_forward_decay.argtypes = [P] * 8 + [P, ctypes.c_int, ctypes.c_int] + \
+                    [P] * 5 + [P, ctypes.c_int, ctypes.c_int]
+                lib.sdm_oracle_forward_decay.restype = ctypes.c_int
             _libs[so] = lib
         return _libs[so]
 
@@ -117,6 +121,46 @@ def forward(inp: Dict[str, np.ndarray], dims: Dict[str, int], t_begin: int = 0,
                                 _ptr(M), _ptr(o), _ptr(_dims(dims)), int(t_begin), int(t_end),
                                 _ptr(iw), _ptr(ww), _ptr(ir), _ptr(wr), _ptr(fl), _ptr(hs), nh,
                                 int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the dimensions or ran out of memory")
+    return out
+
+
+def forward_decay(inp: Dict[str, np.ndarray], dims: Dict[str, int], t_begin: int = 0,
+                  t_end: Optional[int] = None, heads: Optional[Sequence[int]] = None,
+                  nthreads: int = 1, lists: bool = False, M=None, so: Optional[str] = None
+                  ) -> Dict[str, np.ndarray]:
+    """The forward pass with the Raven page's selective-decay write
+    (sdm_oracle_forward_decay): inp as for forward with 'a' [B,H,T] (the decay
+    rate a_t <= 0) in place of alpha and beta.  w_w holds the normalised
+    router weights."""
+    lib = load(so)
+    T = dims['T']
+    t_end = T if t_end is None else t_end
+    q, k, v, a = _f32(inp['q']), _f32(inp['k']), _f32(inp['v']), _f32(inp['a'])
+    C1, C2 = _f32(inp['C1']), _f32(inp['C2'])
+    if M is None:
+        M = _f32(inp['M0']).copy()
+    B, H, dv = dims['B'], dims['H'], dims['d_v']
+    o = np.zeros((B, H, T, dv), dtype=np.float32)
+    out = {'o': o, 'M': M}
+    iw = ww = ir = wr = fl = None
+    if lists:
+        iw = np.full((B, H, T, dims['W']), -1, dtype=np.int64)
+        ww = np.zeros((B, H, T, dims['W']), dtype=np.float64)
+        ir = np.full((B, H, T, dims['R']), -1, dtype=np.int64)
+        wr = np.zeros((B, H, T, dims['R']), dtype=np.float64)
+        fl = np.zeros((B, H, T), dtype=np.uint8)
+        out.update(idx_w=iw, w_w=ww, idx_r=ir, w_r=wr, flags=fl)
+    hs = None
+    nh = 0
+    if heads is not None:
+        hs = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+        nh = int(hs.size)
+    rc = lib.sdm_oracle_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(C1), _ptr(C2),
+                                      _ptr(M), _ptr(o), _ptr(_dims(dims)), int(t_begin),
+                                      int(t_end), _ptr(iw), _ptr(ww), _ptr(ir), _ptr(wr), _ptr(fl),
+                                      _ptr(hs), nh, int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the dimensions or ran out of memory")
     return out

@@ -53,6 +53,7 @@
 
 typedef struct {
   int B, H, T, d_qk, d_v, n_sub, k, W, R;
+  int rule; /* write rule: 0 = gated delta (item 3), 1 = selective decay (Raven) */
 } odims_t;
 
 typedef struct {
@@ -177,6 +178,32 @@ typedef struct {
   uint8_t* flags;
 } head_io_t;
 
+/*
+ * The selective-decay write of the Raven page ("Raven - Modelado de Secuencias
+ * de Alta Recuperacion con Enrutamiento de Memoria Dispersa", section 2.2),
+ * on the slots the product keys selected: the router weights are the sigmoid
+ * of the W selected float32 scores normalised to sum 1 (reading: the page
+ * normalises the kept sigmoid scores; dividing by their sum is the plainest
+ * form), and each selected row decays toward v_t by exp(a_t r_i):
+ *     M[i] = exp(a_t r_i) M[i] + (1 - exp(a_t r_i)) v_t;
+ * unselected rows stay frozen.  Float64, rounded to float32.  ww receives r.
+ */
+static void decay_write(float* M, const int64_t* ws, const float* sw, double* ww, int W, int dv,
+                        double at, const float* vt) {
+  double z = 0.0;
+  for (int j = 0; j < W; ++j) {
+    ww[j] = 1.0 / (1.0 + exp(-(double)sw[j]));
+    z += ww[j];
+  }
+  for (int j = 0; j < W; ++j) ww[j] /= z;
+  for (int j = 0; j < W; ++j) {
+    float* row = M + (size_t)ws[j] * dv;
+    const double dcy = exp(at * ww[j]);
+    for (int col = 0; col < dv; ++col)
+      row[col] = (float)(dcy * (double)row[col] + (1.0 - dcy) * (double)vt[col]);
+  }
+}
+
 static int forward_head(const head_io_t* io, const odims_t* d, int t0, int t1) {
   scratch_t w;
   if (scratch_init(&w, d) != 0) { scratch_free(&w); return -1; }
@@ -184,17 +211,21 @@ static int forward_head(const head_io_t* io, const odims_t* d, int t0, int t1) {
   int64_t* ws = (int64_t*)malloc(sizeof(int64_t) * (size_t)(d->W + d->R));
   double* ww = (double*)malloc(sizeof(double) * (size_t)(d->W + d->R));
   double* acc = (double*)malloc(sizeof(double) * (size_t)dv);
-  if (!ws || !ww || !acc) { free(ws); free(ww); free(acc); scratch_free(&w); return -1; }
+  float* sw = (float*)malloc(sizeof(float) * (size_t)d->W);
+  if (!ws || !ww || !acc || !sw) {
+    free(ws); free(ww); free(acc); free(sw); scratch_free(&w); return -1;
+  }
   int64_t* rs = ws + d->W;
   double* rw = ww + d->W;
   for (int t = t0; t < t1; ++t) {
     /* write selection from k'_t, read selection from q'_t (item 2) */
-    int fl = select_side(io->k + (size_t)t * dq, io->C1, io->C2, d, d->W, &w, ws, ww, NULL, 0);
+    int fl = select_side(io->k + (size_t)t * dq, io->C1, io->C2, d, d->W, &w, ws, ww, sw, 0);
     fl |= select_side(io->q + (size_t)t * dq, io->C1, io->C2, d, d->R, &w, rs, rw, NULL, 3);
-    const double a = (double)io->alpha[t], be = (double)io->beta[t];
+    const double a = (double)io->alpha[t], be = io->beta ? (double)io->beta[t] : 0.0;
     const float* vt = io->v + (size_t)t * dv;
+    if (d->rule == 1) decay_write(io->M, ws, sw, ww, d->W, dv, a, vt);
     /* gated delta write on the W selected slots (item 3) */
-    for (int j = 0; j < d->W; ++j) {
+    for (int j = 0; d->rule == 0 && j < d->W; ++j) {
       float* row = io->M + (size_t)ws[j] * dv;
       const double c = be * ww[j];
       for (int col = 0; col < dv; ++col) {
@@ -216,7 +247,7 @@ static int forward_head(const head_io_t* io, const odims_t* d, int t0, int t1) {
     if (io->w_r) memcpy(io->w_r + (size_t)t * d->R, rw, sizeof(double) * (size_t)d->R);
     if (io->flags) io->flags[t] = (uint8_t)fl;
   }
-  free(ws); free(ww); free(acc);
+  free(ws); free(ww); free(acc); free(sw);
   scratch_free(&w);
   return 0;
 }
@@ -262,7 +293,7 @@ static void* worker(void* arg) {
     io.k = J->k + tq * d->d_qk;
     io.v = J->v + tq * d->d_v;
     io.alpha = J->alpha + tq;
-    io.beta = J->beta + tq;
+    io.beta = J->beta ? J->beta + tq : NULL;
     io.C1 = J->C1 + (size_t)h * d->n_sub * dh;
     io.C2 = J->C2 + (size_t)h * d->n_sub * dh;
     io.M = J->M + (size_t)bh * N * d->d_v;
@@ -333,7 +364,7 @@ int sdm_oracle_select(const float* x, const float* C1, const float* C2, const in
                       int n_sel, int64_t* slots, double* weights, float* scores, int* flag) {
   odims_t d;
   d.B = 1; d.H = 1; d.T = 1; d.d_qk = dims[3]; d.d_v = 1; d.n_sub = dims[5]; d.k = dims[6];
-  d.W = n_sel; d.R = n_sel;
+  d.W = n_sel; d.R = n_sel; d.rule = 0;
   if (!dims_ok(&d)) return -1;
   scratch_t w;
   if (scratch_init(&w, &d) != 0) { scratch_free(&w); return -1; }
@@ -341,4 +372,43 @@ int sdm_oracle_select(const float* x, const float* C1, const float* C2, const in
   if (flag) *flag = f;
   scratch_free(&w);
   return 0;
+}
+
+/*
+ * The forward pass with the Raven page's selective-decay write in place of the
+ * gated delta write (see decay_write): same selection, read, layouts and
+ * optional outputs as sdm_oracle_forward, with a [B][H][T] (a_t <= 0, the
+ * decay rate) in place of alpha and no beta.  w_w receives the normalised
+ * router weights r.
+ */
+int sdm_oracle_forward_decay(const float* q, const float* k, const float* v, const float* a,
+                             const float* C1, const float* C2, float* M, float* o,
+                             const int* dims, int t_begin, int t_end, int64_t* idx_w, double* w_w,
+                             int64_t* idx_r, double* w_r, uint8_t* flags, const int32_t* heads,
+                             int n_heads, int nthreads) {
+  job_t J;
+  memset(&J, 0, sizeof(J));
+  J.d.B = dims[0]; J.d.H = dims[1]; J.d.T = dims[2]; J.d.d_qk = dims[3]; J.d.d_v = dims[4];
+  J.d.n_sub = dims[5]; J.d.k = dims[6]; J.d.W = dims[7]; J.d.R = dims[8];
+  J.d.rule = 1;
+  if (!dims_ok(&J.d) || t_begin < 0 || t_end > J.d.T || t_begin > t_end) return -1;
+  J.q = q; J.k = k; J.v = v; J.alpha = a; J.beta = NULL; J.C1 = C1; J.C2 = C2;
+  J.M = M; J.o = o; J.idx_w = idx_w; J.w_w = w_w; J.idx_r = idx_r; J.w_r = w_r;
+  J.flags = flags;
+  J.t0 = t_begin; J.t1 = t_end;
+  J.heads = heads;
+  J.n_heads = heads ? n_heads : J.d.B * J.d.H;
+  pthread_mutex_init(&J.mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > J.n_heads) nthreads = J.n_heads > 0 ? J.n_heads : 1;
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!th) return -1;
+  int started = 0;
+  for (int i = 0; i < nthreads; ++i)
+    if (pthread_create(&th[i], NULL, worker, &J) == 0) ++started;
+  if (started == 0) worker(&J);
+  for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+  free(th);
+  pthread_mutex_destroy(&J.mu);
+  return J.err ? -1 : 0;
 }

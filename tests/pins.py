@@ -16,6 +16,10 @@ build) and raises AssertionError when the oracle disagrees with:
   * invariants: unselected rows stay bit-identical; splitting the time axis
     with the table carried over gives bit-identical results;
   * W = R = N (k = n): a dense all-slot gated delta update written with numpy;
+  * the selective-decay write (the Raven page's rule on the same selection):
+    a = 0 freezes every row, a very negative overwrites with v_t, a single slot
+    follows e^{a t} m_0 + (1 - e^{a t}) v, router weights are normalised
+    sigmoids, and one step from a known table moves only the selected rows;
   * the near-tie flags, from their definition in the workload specification (a
     float64 gap below 1e-5 relative at the W-th/(W+1)-th (R-th/(R+1)-th)
     candidate, or at a half's k-th/(k+1)-th row): hand-built score tables whose
@@ -369,8 +373,94 @@ def pin_near_tie_flags_float64_gap(so=None):
     assert flag == 1, flag
 
 
+# ---------------------------------------------------------------- selective decay
+# The Raven page's write rule on the product-key selection (oracle.forward_decay):
+# r = sigmoid(score) normalised over the W selected slots; M[i] = exp(a r_i) M[i]
+# + (1 - exp(a r_i)) v_t on the selected rows only.
+def _decay_inp(rng, d, a):
+    inp = _rand_inputs(rng, d, m0_scale=1.0)
+    inp['a'] = (np.full(inp['alpha'].shape, a) if np.isscalar(a) else a).astype(np.float32)
+    return inp
+
+
+def pin_decay_frozen_and_overwrite(so=None):
+    """a = 0: exp(0) = 1, every row frozen (bit-identical).  a = -1e4 with W = R = 1
+    (r = 1, exp(-1e4) = 0 in float64) and q' = k': the written row becomes v_t
+    exactly and the same step's read returns it."""
+    rng = np.random.default_rng(31)
+    d = _dims(B=1, H=2, T=30, d_qk=8, d_v=4, n_sub=5, k=3, W=4, R=3)
+    inp = _decay_inp(rng, d, 0.0)
+    out = oracle.forward_decay(inp, d, so=so)
+    assert np.array_equal(out['M'], inp['M0'])
+    d1 = _dims(B=1, H=2, T=30, d_qk=6, d_v=5, n_sub=6, k=2, W=1, R=1)
+    inp = _decay_inp(rng, d1, -1e4)
+    inp['q'] = inp['k'].copy()
+    out = oracle.forward_decay(inp, d1, so=so)
+    assert np.array_equal(out['o'], inp['v'])
+
+
+def pin_decay_single_slot(so=None):
+    """One slot wins every step (W = R = 1, r = 1): m_t = e^a m_{t-1} + (1 - e^a) v,
+    so m_t = e^{a t} m_0 + (1 - e^{a t}) v and o_t = m_t."""
+    n, dh, T = 4, 4, 40
+    d = _dims(T=T, d_qk=2 * dh, d_v=3, n_sub=n, k=2, W=1, R=1)
+    rng = np.random.default_rng(32)
+    C1 = 0.01 * rng.standard_normal((1, n, dh)).astype(np.float32)
+    C2 = 0.01 * rng.standard_normal((1, n, dh)).astype(np.float32)
+    C1[0, 1] = 5.0
+    C2[0, 3] = 5.0
+    keys = (np.abs(rng.standard_normal((1, 1, T, 2 * dh))) + 0.5).astype(np.float32)
+    vv = np.array([2.0, -1.0, 0.25], np.float32)
+    m0 = np.zeros((1, 1, n * n, 3), np.float32)
+    m0[0, 0, 1 * n + 3] = [1.0, 1.0, 1.0]
+    a = np.float32(-0.3)
+    inp = dict(q=keys.copy(), k=keys, v=np.broadcast_to(vv, (1, 1, T, 3)).copy(),
+               a=np.full((1, 1, T), a, np.float32), C1=C1, C2=C2, M0=m0)
+    out = oracle.forward_decay(inp, d, lists=True, so=so)
+    assert (out['idx_w'][0, 0, :, 0] == 1 * n + 3).all()
+    assert (out['w_w'][0, 0, :, 0] == 1.0).all()
+    e = np.exp(float(a) * np.arange(1, T + 1))[:, None]
+    expect = e * m0[0, 0, 1 * n + 3][None, :] + (1.0 - e) * vv[None, :].astype(np.float64)
+    np.testing.assert_allclose(out['o'][0, 0], expect, rtol=1e-5, atol=1e-6)
+
+
+def pin_decay_router_weights(so=None):
+    """r_i / r_j = sigmoid(s_i) / sigmoid(s_j) over the selected float32 scores, sum
+    1; the selection itself is the product-key top-W (same slots as the oracle's
+    selection of that key)."""
+    rng = np.random.default_rng(33)
+    d = _dims(B=1, H=1, T=12, d_qk=8, d_v=4, n_sub=8, k=4, W=6, R=6)
+    inp = _decay_inp(rng, d, -0.5)
+    out = oracle.forward_decay(inp, d, lists=True, so=so)
+    for t in range(12):
+        slots, _, s, _ = oracle.select(inp['k'][0, 0, t], inp['C1'][0], inp['C2'][0], d, 6, so=so)
+        assert out['idx_w'][0, 0, t].tolist() == slots.tolist()
+        sig = 1.0 / (1.0 + np.exp(-s.astype(np.float64)))
+        np.testing.assert_allclose(out['w_w'][0, 0, t], sig / sig.sum(), rtol=1e-12)
+
+
+def pin_decay_one_step_rows(so=None):
+    """One step from a known table: each selected row i becomes
+    exp(a r_i) M0[i] + (1 - exp(a r_i)) v; every other row is unchanged."""
+    rng = np.random.default_rng(34)
+    d = _dims(B=1, H=1, T=1, d_qk=8, d_v=4, n_sub=6, k=3, W=5, R=2)
+    inp = _decay_inp(rng, d, -0.8)
+    out = oracle.forward_decay(inp, d, lists=True, so=so)
+    M0 = inp['M0'][0, 0].astype(np.float64)
+    sel = out['idx_w'][0, 0, 0]
+    r = out['w_w'][0, 0, 0]
+    expect = M0.copy()
+    for i, ri in zip(sel, r):
+        dcy = np.exp(-0.8 * ri)
+        expect[i] = dcy * M0[i] + (1.0 - dcy) * inp['v'][0, 0, 0].astype(np.float64)
+    np.testing.assert_allclose(out['M'][0, 0], expect, rtol=1e-6, atol=1e-7)
+    other = np.setdiff1d(np.arange(36), sel)
+    assert np.array_equal(out['M'][0, 0, other], inp['M0'][0, 0, other])
+
+
 ALL_PINS = [pin_golden, pin_bruteforce_identity, pin_gates_identity,
             pin_overwrite_and_read_after_write, pin_single_slot_recurrence, pin_softmax_weights,
             pin_ties_lowest_index, pin_half_split_and_slot_numbering, pin_untouched_rows,
             pin_streaming, pin_dense_all_slots, pin_near_tie_flags,
-            pin_near_tie_flags_float64_gap]
+            pin_near_tie_flags_float64_gap, pin_decay_frozen_and_overwrite, pin_decay_single_slot,
+            pin_decay_router_weights, pin_decay_one_step_rows]

@@ -79,6 +79,17 @@ MUTANTS = {
     "half-flag-wrong-pair": lambda s: s.replace(
         "near_tie(w->s64_1[w->h1[k - 1].id], w->s64_1[w->h1[k].id])",
         "near_tie(w->s64_1[w->h1[k > 1 ? k - 2 : 0].id], w->s64_1[w->h1[k - 1].id])"),
+    "decay-weights-unnormalised": lambda s: s.replace(
+        "  for (int j = 0; j < W; ++j) ww[j] /= z;\n", ""),
+    "decay-softmax-router": lambda s: s.replace(
+        "    ww[j] = 1.0 / (1.0 + exp(-(double)sw[j]));", "    ww[j] = exp((double)sw[j]);"),
+    "decay-exponent-sign": lambda s: s.replace(
+        "    const double dcy = exp(at * ww[j]);", "    const double dcy = exp(-at * ww[j]);"),
+    "decay-toward-zero": lambda s: s.replace(
+        "      row[col] = (float)(dcy * (double)row[col] + (1.0 - dcy) * (double)vt[col]);",
+        "      row[col] = (float)(dcy * (double)row[col]);"),
+    "decay-ignores-router": lambda s: s.replace(
+        "    const double dcy = exp(at * ww[j]);", "    const double dcy = exp(at);"),
     "fp64-candidate-order": lambda s: s.replace(
         "float s = w->h1[a].s + w->h2[b].s;          /* float32 sum */",
         "float s = (float)(w->s64_1[w->h1[a].id] + w->s64_2[w->h2[b].id]);"),
@@ -115,3 +126,5 @@ def test_mutant_is_caught(name, mutant_dir):
             "sys.exit(1 if bad else 0)\n") % (here, os.path.dirname(here), so)
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
     assert r.returncode != 0, "no pin catches the mutation %r" % name
+    # a pin's assertion catches it (not a crash of the broken copy)
+    assert r.stdout.strip() not in ("", "[]"), r.stderr[-2000:]
