@@ -49,6 +49,7 @@ def mutant_dir():
 
 @pytest.mark.parametrize("name", sorted(GDN_MUTANTS))
 def test_gdn_mutant_is_caught(name, mutant_dir):
+    from test_oracle_mutations import _caught_by_a_pin
     with open(oracle.GDN_SRC) as f:
         src = f.read()
     bad = GDN_MUTANTS[name](src)
@@ -58,17 +59,5 @@ def test_gdn_mutant_is_caught(name, mutant_dir):
     with open(c, "w") as f:
         f.write(bad)
     oracle.compile_source(c, so)
-    here = os.path.dirname(os.path.abspath(__file__))
-    code = ("import sys; sys.path[:0] = [%r, %r]\n"
-            "import gdn_pins\n"
-            "bad = []\n"
-            "for pin in gdn_pins.GDN_PINS:\n"
-            "    try:\n"
-            "        pin(%r)\n"
-            "    except AssertionError:\n"
-            "        bad.append(pin.__name__)\n"
-            "print(bad)\n"
-            "sys.exit(1 if bad else 0)\n") % (here, os.path.dirname(here), so)
-    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
-    assert r.returncode != 0, "no pin catches the mutation %r" % name
-    assert r.stdout.strip() not in ("", "[]"), r.stderr
+    assert _caught_by_a_pin("gdn_pins", [p.__name__ for p in gdn_pins.GDN_PINS], so), \
+        "no pin's assertion catches the mutation %r" % name
