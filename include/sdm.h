@@ -28,7 +28,8 @@
  *      M      [B][H][N][d_v]    float32, N = n_sub^2
  *      o      [B][H][T][d_v]    float32
  *      idx_w / w_w [B][H][T][W] int32 / float32 (idx_r / w_r likewise with R)
- *  - Every device pointer must be 16-byte aligned; outputs must not alias
+ *  - Every device pointer must be 16-byte aligned, except the per-step gate
+ *    arrays (alpha, beta, a), which need 4 bytes; outputs must not alias
  *    inputs or each other.  With T == 0 nothing is enqueued and no pointer is
  *    read (empty tensors may pass NULL).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work
@@ -77,7 +78,7 @@ enum {
   SDM_OK = 0,
   SDM_ERR_NULL = 1,        /* a required pointer is NULL */
   SDM_ERR_DIMS = 2,        /* sizes out of range or inconsistent */
-  SDM_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  SDM_ERR_ALIGN = 3,       /* a pointer is misaligned (16 bytes; 4 for gate arrays) */
   SDM_ERR_WORKSPACE = 4,   /* workspace missing or smaller than sdm_workspace_bytes */
   SDM_ERR_UNSUPPORTED = 5, /* valid sizes this build has no kernel for */
   SDM_ERR_CUDA = 6,        /* a CUDA call failed while enqueueing */
@@ -163,6 +164,24 @@ SDM_API int sdm_step(const void* q, const void* k, const void* v, const float* a
                      const float* beta, const void* C1, const void* C2, float* M_inout,
                      float* o_out, int32_t* idx_w, float* w_w, int32_t* idx_r, float* w_r,
                      const sdm_dims* dims, void* stream);
+
+/*
+ * The forward pass with the Raven page's selective-decay write rule ("Raven -
+ * Modelado de Secuencias de Alta Recuperacion con Enrutamiento de Memoria
+ * Dispersa", section 2.2) in place of the gated delta write, on SDM's
+ * product-key selection: the router weight of write slot i is the sigmoid of
+ * its selected score normalised over the W selected slots, r_i = s(x_i) /
+ * sum_j s(x_j), and each selected row decays toward v_t,
+ *     M[i] = exp(a_t r_i) M[i] + (1 - exp(a_t r_i)) v_t,
+ * unselected rows staying frozen; the read is SDM's (softmax over the R read
+ * scores, after the write).  a [B][H][T] float32 holds the decay rate a_t
+ * (<= 0; 0 freezes).  Everything else, including the workspace
+ * (sdm_workspace_bytes), as sdm_forward.
+ */
+SDM_API int sdm_forward_decay(const void* q, const void* k, const void* v, const float* a,
+                              const void* C1, const void* C2, float* M_inout, float* o_out,
+                              const sdm_dims* dims, void* workspace, size_t ws_bytes,
+                              void* stream);
 
 /*
  * sdm_forward that also records caller-created CUDA events (cudaEvent_t) on

@@ -7,6 +7,7 @@ into pointers and the current CUDA stream.  There is no CPU path: calling
 without the built library, or with CPU tensors, raises.
 """
 from .sdm import (  # noqa: F401
-    SDMError, Dims, LIB_PATH, load_library, workspace_bytes, forward, step, select, recur,
+    SDMError, Dims, LIB_PATH, load_library, workspace_bytes, forward, forward_decay, step, select,
+    recur,
     device_status, make_dims, query_plan, PLAN_FIELDS, gdn_forward, gdn_workspace_bytes, GdnDims,
 )

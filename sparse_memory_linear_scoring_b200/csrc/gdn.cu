@@ -238,9 +238,13 @@ k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float
   for (int c = 0; c < p.nch; ++c) {
     float* st = stg + (STAGES == 2 ? (c & 1) : 0) * sf;
     if (STAGES == 2 && c + 1 < p.nch) {
+      // the other stage was last read in iteration c - 1, before its final barrier
       load(c + 1, stg + ((c + 1) & 1) * sf);
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
+      // one stage: chunk c is loaded here, after iteration c - 1's final
+      // barrier (chunk 0 was loaded above)
+      if (STAGES == 1 && c > 0) load(c, stg);
       asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
@@ -307,10 +311,14 @@ extern "C" int sdm_gdn_forward(const void* q, const void* k, const void* v, cons
   int rc = gdn_plan(dims, &p);
   if (rc != SDM_OK) return rc;
   if (p.T == 0) return SDM_OK;
-  const void* ps[] = {q, k, v, alpha, beta, S_inout, o_out, workspace};
+  const void* ps[] = {q, k, v, S_inout, o_out, workspace};
   for (const void* x : ps) {
     if (!x) return x == workspace ? SDM_ERR_WORKSPACE : SDM_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) & 15) return SDM_ERR_ALIGN;
+  }
+  for (const void* x : {static_cast<const void*>(alpha), static_cast<const void*>(beta)}) {
+    if (!x) return SDM_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) & 3) return SDM_ERR_ALIGN;  // per-step scalars
   }
   if (ws_bytes < p.total) return SDM_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -206,7 +206,7 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
                           int n_sel, const uint32_t* stair, int n_stair, const uint32_t* front,
                           int nf, uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* cell,
                           uint32_t* alt, uint64_t* sel, bool sorted, float* w_out,
-                          uint32_t* slot_out, DevStatus* st, int info) {
+                          uint32_t* slot_out, DevStatus* st, int info, bool sigmoid_w = false) {
   const int lane = threadIdx.x & 31;
   if (c1 < p.k || c1 > p.C || c2 < p.k || c2 > p.C) {
     if (lane == 0) dev_flag(st, SDM_DEV_CAPACITY, info);
@@ -338,12 +338,15 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
     __syncwarp();
     warp_sort_desc(sel, S);
   }
-  // softmax over the selected float32 scores; the best candidate is (0, 0)
+  // softmax over the selected float32 scores (the best candidate is (0, 0));
+  // with sigmoid_w, the router weights of the selective-decay rule instead:
+  // sigmoid of each selected score, normalised to sum 1
   const float m = key_val(h1[0]) + key_val(h2[0]);
   float* ex = reinterpret_cast<float*>(cand);  // free again (n_sel <= Sc)
   float zs = 0.f;
   for (int i = lane; i < n_sel; i += 32) {
-    const float e = expf(key_val(sel[i]) - m);
+    const float s = key_val(sel[i]);
+    const float e = sigmoid_w ? 1.f / (1.f + expf(-s)) : expf(s - m);
     ex[i] = e;
     zs += e;
   }

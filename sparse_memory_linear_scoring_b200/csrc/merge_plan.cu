@@ -27,7 +27,9 @@
 // step's write before its read).  A record is
 //   int4 {slot, (step_in_chunk << 1) | is_read, f1, f2}
 // with, for a write, f1 = alpha_t * (1 - c), f2 = c = beta_t * w_i (the update
-// is then M = f1 * M + f2 * v_t); for a read, f1 = u_r.  The per-(head, block)
+// is then M = f1 * M + f2 * v_t); for a read, f1 = u_r.  Under the selective-
+// decay write rule (the Raven page, section 2.2: router weight r_i, decay
+// rate a_t), f1 = exp(a_t r_i) and f2 = 1 - f1.  The per-(head, block)
 // bucket starts (NB + 1 of them) go to roff.
 #include "merge_dev.cuh"
 
@@ -89,7 +91,7 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
               io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
               side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, cell, alt, sel,
-              io.sorted != 0, w_out, s_out, st, int(hr));
+              io.sorted != 0, w_out, s_out, st, int(hr), p.rule == 1 && side == 0);
   }
 }
 
@@ -210,7 +212,7 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
         } else {
           w[i] = io.ww[(lrow0 + tl) * p.W + j];
           al[i] = io.alpha[trow0 + tl];
-          be[i] = io.beta[trow0 + tl];
+          be[i] = p.rule == 1 ? 0.f : io.beta[trow0 + tl];
         }
       }
     }
@@ -244,6 +246,11 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
       if (is_read) {
         r.z = __float_as_int(w[i]);
         r.w = 0;
+      } else if (p.rule == 1) {
+        // selective decay: M = e^{a r} M + (1 - e^{a r}) v, with a in alpha
+        const float d = expf(al[i] * w[i]);
+        r.z = __float_as_int(d);
+        r.w = __float_as_int(1.f - d);
       } else {
         const float c = be[i] * w[i];
         r.z = __float_as_int(al[i] * (1.f - c));

@@ -196,6 +196,17 @@ static int check_ptrs(std::initializer_list<const void*> ps) {
   return worst;
 }
 
+// Per-step scalars (alpha, beta, a) are read one float at a time: 4-byte
+// alignment is enough, so a time slice of a caller's gate tensor can be passed
+// as it is.
+static int check_gates(std::initializer_list<const void*> ps) {
+  for (const void* q : ps) {
+    if (!q) return SDM_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(q) & 3) return SDM_ERR_ALIGN;
+  }
+  return SDM_OK;
+}
+
 static cudaError_t score_chunk(const Plan& p, const Carve& c, const void* q, const void* k,
                                const void* C1, const void* C2, int t0, int tlen, cudaStream_t s) {
   cudaError_t e;
@@ -229,13 +240,16 @@ int sdm::forward_with_budget(const void* q, const void* k, const void* v, const 
                              const float* beta, const void* C1, const void* C2, float* M_inout,
                              float* o_out, const sdm_dims* dims, void* workspace,
                              size_t ws_bytes, void* stream, void* const* events, int n_events,
-                             size_t chunk_budget) {
+                             size_t chunk_budget, int rule) {
   Plan p;
   int rc = make_plan(dims, &p, chunk_budget);
   if (rc != SDM_OK) return rc;
+  p.rule = rule;
   if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
-  rc = check_ptrs({q, k, v, alpha, beta, C1, C2, M_inout, o_out, workspace});
+  rc = check_ptrs({q, k, v, C1, C2, M_inout, o_out, workspace});
   if (rc != SDM_OK) return rc == SDM_ERR_NULL && !workspace ? SDM_ERR_WORKSPACE : rc;
+  // the selective-decay rule has no beta
+  if ((rc = check_gates({alpha, rule == 1 ? alpha : beta})) != SDM_OK) return rc;
   if (ws_bytes < p.total) return SDM_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Carve c = carve(p, workspace);
@@ -297,6 +311,14 @@ extern "C" int sdm_forward_timed(const void* q, const void* k, const void* v, co
                              ws_bytes, stream, events, n_events, kChunkBudget);
 }
 
+extern "C" int sdm_forward_decay(const void* q, const void* k, const void* v, const float* a,
+                                 const void* C1, const void* C2, float* M_inout, float* o_out,
+                                 const sdm_dims* dims, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  return forward_with_budget(q, k, v, a, nullptr, C1, C2, M_inout, o_out, dims, workspace,
+                             ws_bytes, stream, nullptr, 0, kChunkBudget, 1);
+}
+
 extern "C" int sdm_query_plan(const sdm_dims* dims, int64_t* out, int n) {
   Plan p;
   const int rc = make_plan(dims, &p);
@@ -346,8 +368,9 @@ extern "C" int sdm_recur(const void* v, const float* alpha, const float* beta,
   int rc = make_plan(dims, &p);
   if (rc != SDM_OK) return rc;
   if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
-  rc = check_ptrs({v, alpha, beta, idx_w, w_w, idx_r, w_r, M_inout, o_out, workspace});
+  rc = check_ptrs({v, idx_w, w_w, idx_r, w_r, M_inout, o_out, workspace});
   if (rc != SDM_OK) return rc == SDM_ERR_NULL && !workspace ? SDM_ERR_WORKSPACE : rc;
+  if ((rc = check_gates({alpha, beta})) != SDM_OK) return rc;
   if (ws_bytes < p.total) return SDM_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Carve c = carve(p, workspace);
@@ -392,7 +415,7 @@ extern "C" const char* sdm_status_string(int status) {
     case SDM_OK: return "ok";
     case SDM_ERR_NULL: return "a required pointer is NULL";
     case SDM_ERR_DIMS: return "sizes out of range or inconsistent";
-    case SDM_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case SDM_ERR_ALIGN: return "a device pointer is misaligned (16 bytes; 4 for gate arrays)";
     case SDM_ERR_WORKSPACE: return "workspace missing or too small";
     case SDM_ERR_UNSUPPORTED: return "valid sizes without a kernel in this build";
     case SDM_ERR_CUDA: return "a CUDA call failed while enqueueing";

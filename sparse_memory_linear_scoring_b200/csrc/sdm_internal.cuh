@@ -56,6 +56,7 @@ struct Plan {
   int B, H, T, dqk, dh, dv, n, k, W, R, dtype;
   int BH;
   long long N;
+  int rule;    // write rule: 0 gated delta (alpha, beta), 1 selective decay (a)
   int tc;      // scoring mode: 0 CUDA cores, 1 tensor cores + in-kernel selection,
                // 2 tensor-core filter + survivor top-k (score_tc_mode)
   int C;       // survivor capacity per half-row
@@ -92,7 +93,8 @@ int make_plan(const sdm_dims* d, Plan* p, size_t chunk_budget = kChunkBudget);
 int forward_with_budget(const void* q, const void* k, const void* v, const float* alpha,
                         const float* beta, const void* C1, const void* C2, float* M_inout,
                         float* o_out, const sdm_dims* dims, void* workspace, size_t ws_bytes,
-                        void* stream, void* const* events, int n_events, size_t chunk_budget);
+                        void* stream, void* const* events, int n_events, size_t chunk_budget,
+                        int rule = 0);
 
 // ---- device helpers ---------------------------------------------------------
 __device__ __forceinline__ uint32_t f2ord(float v) {

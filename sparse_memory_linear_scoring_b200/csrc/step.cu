@@ -341,10 +341,14 @@ extern "C" int sdm_step(const void* q, const void* k, const void* v, const float
   size_t smem = 0;
   if (!step_supported(p, &smem)) return SDM_ERR_UNSUPPORTED;
   if (p.T == 0) return SDM_OK;  // nothing to do; no pointer is read
-  const void* ps[] = {q, k, v, alpha, beta, C1, C2, M_inout, o_out};
+  const void* ps[] = {q, k, v, C1, C2, M_inout, o_out};
   for (const void* x : ps) {
     if (!x) return SDM_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) & 15) return SDM_ERR_ALIGN;
+  }
+  for (const void* x : {static_cast<const void*>(alpha), static_cast<const void*>(beta)}) {
+    if (!x) return SDM_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) & 3) return SDM_ERR_ALIGN;  // per-step scalars
   }
   const int nl = (idx_w != nullptr) + (w_w != nullptr) + (idx_r != nullptr) + (w_r != nullptr);
   if (nl != 0 && nl != 4) return SDM_ERR_NULL;

@@ -70,6 +70,8 @@ def load_library():
             lib.sdm_gdn_workspace_bytes.restype = S
             lib.sdm_gdn_forward.argtypes = [P] * 7 + [ctypes.POINTER(GdnDims), P, S, P]
             lib.sdm_gdn_forward.restype = ctypes.c_int
+            lib.sdm_forward_decay.argtypes = [P] * 8 + [DP, P, S, P]
+            lib.sdm_forward_decay.restype = ctypes.c_int
             lib.sdm_step.argtypes = [P] * 13 + [DP, P]
             lib.sdm_step.restype = ctypes.c_int
             lib.sdm_version.argtypes = []
@@ -240,6 +242,30 @@ def forward(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
     _check(lib.sdm_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(C1), _ptr(C2),
                            _ptr(M), _ptr(o), ctypes.byref(dims), _ptr(ws), _nbytes(ws),
                            _stream(dev, stream)))
+    return o
+
+
+def forward_decay(q, k, v, a, C1, C2, M, *, topk: int, W: int, R: int,
+                  o: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """SDM with the Raven page's selective-decay write (sdm_forward_decay): a
+    [B,H,T] float32 decay rates (<= 0) in place of alpha and beta; otherwise as
+    forward.  Returns o; M is updated in place."""
+    B, H, T, d_qk, n_sub, dt = _check_inputs(q, k, v, C1, C2, a, None)
+    d_v = v.shape[-1]
+    _expect(M, "M", (B, H, n_sub * n_sub, d_v), (torch.float32,))
+    if o is not None:
+        _expect(o, "o", (B, H, T, d_v), (torch.float32,))
+    dev = _dev(q, k, v, a, C1, C2, M, *([o] if o is not None else []))
+    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, W, R, dt)
+    if o is None:
+        o = torch.empty(B, H, T, d_v, dtype=torch.float32, device=dev)
+    _no_alias([("M", M), ("o", o)], [("q", q), ("k", k), ("v", v), ("a", a), ("C1", C1),
+                                     ("C2", C2)])
+    ws = _workspace(dims, dev, workspace)
+    _check(load_library().sdm_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(C1),
+                                            _ptr(C2), _ptr(M), _ptr(o), ctypes.byref(dims),
+                                            _ptr(ws), _nbytes(ws), _stream(dev, stream)))
     return o
 
 

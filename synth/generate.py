@@ -49,6 +49,7 @@ _MIX2_S = _s64(_MIX2)
 TID_Q, TID_K, TID_V, TID_ALPHA, TID_BETA, TID_C1, TID_C2, TID_M0 = 1, 2, 3, 4, 5, 6, 7, 8
 TID_PATTERN, TID_PICK, TID_NOISE = 9, 10, 11
 TID_GDN_Q, TID_GDN_K, TID_GDN_S0 = 12, 13, 14
+TID_DECAY = 15
 
 
 def _mix_int(z: int) -> int:
@@ -277,3 +278,14 @@ def gen_gdn_inputs(cfg: SDMConfig, d_k: Optional[int] = None, seed: int = 0, dev
     else:
         out['S0'] = torch.zeros(cfg.B, cfg.H, cfg.d_v, d_k, dtype=torch.float32, device=device)
     return out
+
+
+def gen_decay_rate(cfg: SDMConfig, seed: int = 0, device: str = 'cpu', b0: int = 0,
+                   t_end: Optional[int] = None) -> torch.Tensor:
+    """Decay rates of the selective-decay write rule, [B,H,T] float32:
+    a_t = -softplus(N(0, 1)) (negative, as a Mamba-2 style input-dependent rate;
+    the Raven page gives no distribution), computed in float64."""
+    T = cfg.T if t_end is None else t_end
+    z = _normals(cfg, seed, TID_DECAY, list(range(b0, b0 + cfg.B)), list(range(cfg.H)), (T,),
+                 device)
+    return (-torch.nn.functional.softplus(z)).to(torch.float32)

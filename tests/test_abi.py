@@ -82,7 +82,8 @@ def test_pointer_checks(lib):
         a = list(args)
         a[i] = None
         assert lib.sdm_forward(*a, ctypes.byref(dims), fake, need, None) == ERR_NULL
-        a[i] = ctypes.c_void_p((1 << 20) + 4)
+        gate = i in (3, 4)                   # alpha, beta: 4-byte alignment suffices
+        a[i] = ctypes.c_void_p((1 << 20) + (2 if gate else 4))
         assert lib.sdm_forward(*a, ctypes.byref(dims), fake, need, None) == ERR_ALIGN
     sel = [fake] * 8
     assert lib.sdm_select(*sel[:4], None, *sel[5:], ctypes.byref(dims), fake, need, None) == ERR_NULL
