@@ -21,9 +21,9 @@
 // not depend on S_0 (U~, W, P, Q~ = diag(exp(g)) Q, K~ = diag(exp(g_last - g)) K,
 // exp(g_last)); rows past a partial last chunk are zero.  W, Q~ and P are
 // stored transposed (step index fastest), which is how the scan reads them.
-// k_gdn_scan then walks the chunks of one head in order for a block of RB rows
-// of S -- rows are independent under this rule -- and writes o and the final
-// S.  Everything is float32 on CUDA cores; the state stays in shared memory.
+// k_gdn_scan then walks the chunks of one head in order for a block of RB = 4
+// rows of S -- rows are independent under this rule -- and writes o and the
+// final S.  Everything is float32 on CUDA cores; the state stays in shared memory.
 #include <string.h>
 
 #include "sdm_internal.cuh"
@@ -32,7 +32,7 @@ namespace sdm {
 
 constexpr int kGdnC = 64;          // steps per chunk
 constexpr int kGdnThreads = 256;
-constexpr int kGdnRB = 8;          // rows of S per scan CTA
+constexpr int kGdnRB = 4;          // rows of S per scan CTA (two warps per row)
 
 struct GdnPlan {
   int B, H, T, dk, dv, dtype, BH, nch;
@@ -225,7 +225,7 @@ k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float
     }
     for (int i = tid; i < kGdnC * kGdnC / 4; i += kGdnThreads)
       cp16(st + 3 * kGdnC * dk + 4 * i, src + p.oP + 4 * i);
-    // U~ columns i0 .. i0 + RB of every row: RB = 8 floats = two 16-byte pieces
+    // U~ columns i0 .. i0 + RB of every row: RB floats in 16-byte pieces
     for (int i = tid; i < kGdnC * (kGdnRB / 4); i += kGdnThreads) {
       const int t = i / (kGdnRB / 4), h4 = i - t * (kGdnRB / 4);
       cp16(st + 3 * kGdnC * dk + kGdnC * kGdnC + t * kGdnRB + 4 * h4,
@@ -254,27 +254,20 @@ k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float
     const float* Pt = st + 3 * kGdnC * dk;  // [C (j)][C (t)]
     const float* Ut = Pt + kGdnC * kGdnC;   // [C][RB]
     const float gl = Ut[kGdnC * kGdnRB];
-    // warp w takes row r = w of the block; lane l takes steps l and l + 32.
+    // warps 2r and 2r + 1 take row r of the block; each lane one step t.
     // U[t][r] = U~[t][r] - W[t] . S[r];  o[t][r] = Q~[t] . S[r] + sum_{j<=t} P[t][j] U[j][r]
-    const int r = tid >> 5, lane = tid & 31;
-    float su0 = 0.f, su1 = 0.f, sq0 = 0.f, sq1 = 0.f;
+    const int lane = tid & 31, r = tid >> 6, ts = ((tid >> 5) & 1) * 32 + lane;
+    float su = 0.f, sq = 0.f;
     for (int e = 0; e < dk; ++e) {
       const float sv = Ss[r * dk + e];
-      su0 = fmaf(Wt[e * kGdnC + lane], sv, su0);
-      su1 = fmaf(Wt[e * kGdnC + lane + 32], sv, su1);
-      sq0 = fmaf(Qt[e * kGdnC + lane], sv, sq0);
-      sq1 = fmaf(Qt[e * kGdnC + lane + 32], sv, sq1);
+      su = fmaf(Wt[e * kGdnC + ts], sv, su);
+      sq = fmaf(Qt[e * kGdnC + ts], sv, sq);
     }
-    Us[lane * kGdnRB + r] = Ut[lane * kGdnRB + r] - su0;
-    Us[(lane + 32) * kGdnRB + r] = Ut[(lane + 32) * kGdnRB + r] - su1;
+    Us[ts * kGdnRB + r] = Ut[ts * kGdnRB + r] - su;
     __syncthreads();
-    for (int jj = 0; jj < kGdnC; ++jj) {  // P is zero above its diagonal
-      const float u = Us[jj * kGdnRB + r];
-      sq0 = fmaf(Pt[jj * kGdnC + lane], u, sq0);
-      sq1 = fmaf(Pt[jj * kGdnC + lane + 32], u, sq1);
-    }
-    Os[lane * kGdnRB + r] = sq0;
-    Os[(lane + 32) * kGdnRB + r] = sq1;
+    const int jend = (ts & ~31) + 32;  // P is zero above its diagonal
+    for (int jj = 0; jj < jend; ++jj) sq = fmaf(Pt[jj * kGdnC + ts], Us[jj * kGdnRB + r], sq);
+    Os[ts * kGdnRB + r] = sq;
     // S[r] = exp(g_last) S[r] + sum_t U[t][r] K~[t]
     for (int i = tid; i < kGdnRB * dk; i += kGdnThreads) {
       const int rr = i / dk, e = i - rr * dk;

@@ -17,6 +17,12 @@ namespace sdm {
 constexpr uint32_t kEmpty = 0xffffffffu;
 constexpr uint32_t kInvalid = 0xffffffffu;
 
+// A sorted half-list entry in shared memory: the float32 score's bits in the
+// high word, the codebook row in the low word (only read back, never ordered
+// as an integer).
+__device__ __forceinline__ float hval(uint64_t e) { return __uint_as_float(uint32_t(e >> 32)); }
+__device__ __forceinline__ uint32_t hrow(uint64_t e) { return uint32_t(e); }
+
 __host__ __device__ inline int p2(int x) {
   int p = 2;
   while (p < x) p <<= 1;
@@ -39,7 +45,7 @@ __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   L.Ss = p2(p.W > p.R ? p.W : p.R);
   L.warps = warps;
   size_t o = 0;
-  L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR) * 4);
+  L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR + 2 * p.k) * 4);
   L.uni = o;
   // h1, h2 [Sk], sel [Ss] (64-bit); cand, cell [Sc], select scratch [2 Sc] (32-bit)
   L.per_warp = size_t(2 * L.Sk + L.Ss) * 8 + size_t(4 * L.Sc) * 4;
@@ -62,8 +68,8 @@ __device__ inline void merge_full(const uint64_t* h1, const uint64_t* h2, int k,
     int cnt = 0;
     for (int i = lane; i < kk; i += 32) {
       const int a = i / k, b = i - a * k;
-      const float v = key_val(h1[a]) + key_val(h2[b]);
-      const uint32_t slot = key_idx(h1[a]) * uint32_t(n) + key_idx(h2[b]);
+      const float v = hval(h1[a]) + hval(h2[b]);
+      const uint32_t slot = hrow(h1[a]) * uint32_t(n) + hrow(h2[b]);
       cnt += make_key(v, slot) >= probe;
     }
     cnt = __reduce_add_sync(0xffffffffu, cnt);
@@ -77,8 +83,8 @@ __device__ inline void merge_full(const uint64_t* h1, const uint64_t* h2, int k,
     bool take = false;
     if (i < kk) {
       const int a = i / k, b = i - a * k;
-      const float v = key_val(h1[a]) + key_val(h2[b]);
-      const uint32_t slot = key_idx(h1[a]) * uint32_t(n) + key_idx(h2[b]);
+      const float v = hval(h1[a]) + hval(h2[b]);
+      const uint32_t slot = hrow(h1[a]) * uint32_t(n) + hrow(h2[b]);
       key = make_key(v, slot);
       take = key >= prefix;
     }
@@ -204,7 +210,7 @@ __device__ inline uint32_t warp_select32(const uint32_t* cand, int n, int r, uin
 // Selection order is unspecified unless `sorted` is set (then rank order).
 __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
                           int n_sel, const uint32_t* stair, int n_stair, const uint32_t* front,
-                          int nf, uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* cell,
+                          int nf, const int* ediv, uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* cell,
                           uint32_t* alt, uint64_t* sel, bool sorted, float* w_out,
                           uint32_t* slot_out, DevStatus* st, int info, bool sigmoid_w = false) {
   const int lane = threadIdx.x & 31;
@@ -216,8 +222,8 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   }
   for (int i = lane; i < p.k; i += 32) {
     const uint2 a = sv1[i], b = sv2[i];
-    h1[i] = make_key(__uint_as_float(a.x), a.y);
-    h2[i] = make_key(__uint_as_float(b.x), b.y);
+    h1[i] = (uint64_t(a.x) << 32) | a.y;
+    h2[i] = (uint64_t(b.x) << 32) | b.y;
   }
   __syncwarp();
   const uint32_t n = uint32_t(p.n);
@@ -226,8 +232,8 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   // columns, and float32 addition is monotone).
   uint32_t lb = 0;
   for (int d = lane + 1; d <= p.k; d += 32) {
-    const int e = (n_sel + d - 1) / d;
-    if (e <= p.k) lb = max(lb, f2ord(key_val(h1[d - 1]) + key_val(h2[e - 1])));
+    const int e = ediv[d - 1];  // ceil(n_sel / d)
+    if (e <= p.k) lb = max(lb, f2ord(hval(h1[d - 1]) + hval(h2[e - 1])));
   }
   lb = __reduce_max_sync(0xffffffffu, lb);
   // candidates: the staircase cells scoring >= lb (ordered 32-bit images of the
@@ -239,7 +245,7 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
     uint32_t x = 0, ab = 0;
     if (i < n_stair) {
       ab = stair[i];
-      x = f2ord(key_val(h1[ab & 0xffff]) + key_val(h2[ab >> 16]));
+      x = f2ord(hval(h1[ab & 0xffff]) + hval(h2[ab >> 16]));
     }
     const bool keep = i < n_stair && x >= lb;
     const unsigned m = __ballot_sync(0xffffffffu, keep);
@@ -265,7 +271,7 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   bool bad = false;
   for (int i = lane; i < nf; i += 32) {
     const uint32_t ab = front[i];
-    bad |= f2ord(key_val(h1[ab & 0xffff]) + key_val(h2[ab >> 16])) >= vstar;
+    bad |= f2ord(hval(h1[ab & 0xffff]) + hval(h2[ab >> 16])) >= vstar;
   }
   bool is_sorted = false;
   if (__any_sync(0xffffffffu, bad) || n_gt + n_eq != n_sel) {
@@ -283,8 +289,8 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
       uint32_t slot = 0;
       if (i < kk) {
         const int a = i / p.k, b = i - a * p.k;
-        tie = f2ord(key_val(h1[a]) + key_val(h2[b])) == vstar;
-        slot = key_idx(h1[a]) * n + key_idx(h2[b]);
+        tie = f2ord(hval(h1[a]) + hval(h2[b])) == vstar;
+        slot = hrow(h1[a]) * n + hrow(h2[b]);
       }
       const unsigned m = __ballot_sync(0xffffffffu, tie);
       const int pos = n_tie + __popc(m & lanemask_lt());
@@ -309,7 +315,7 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
           const uint32_t ab = cell[i];
           const uint64_t a = h1[ab & 0xffff], b = h2[ab >> 16];
           sel[base + __popc(m & lanemask_lt())] =
-              (uint64_t(cand[i]) << 32) | uint64_t(~(key_idx(a) * n + key_idx(b)));
+              (uint64_t(cand[i]) << 32) | uint64_t(~(hrow(a) * n + hrow(b)));
         }
         base += __popc(m);
       }
@@ -326,7 +332,7 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
         const uint32_t ab = cell[i];
         const uint64_t a = h1[ab & 0xffff], b = h2[ab >> 16];
         sel[base + __popc(m & lanemask_lt())] =
-            (uint64_t(cand[i]) << 32) | uint64_t(~(key_idx(a) * n + key_idx(b)));
+            (uint64_t(cand[i]) << 32) | uint64_t(~(hrow(a) * n + hrow(b)));
       }
       base += __popc(m);
     }
@@ -341,7 +347,7 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   // softmax over the selected float32 scores (the best candidate is (0, 0));
   // with sigmoid_w, the router weights of the selective-decay rule instead:
   // sigmoid of each selected score, normalised to sum 1
-  const float m = key_val(h1[0]) + key_val(h2[0]);
+  const float m = hval(h1[0]) + hval(h2[0]);
   float* ex = reinterpret_cast<float*>(cand);  // free again (n_sel <= Sc)
   float zs = 0.f;
   for (int i = lane; i < n_sel; i += 32) {
@@ -362,9 +368,12 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
 
 // Staircase rows a < k with bm(a) = min(k, n_sel / (a+1)) columns, and the
 // frontier cell (a, bm(a)) of each row that stops short of k (rows past the
-// last non-empty one contribute only their first empty cell).  One warp.
-__device__ inline void build_staircase(int k, int n_sel, uint32_t* stair, uint32_t* front) {
+// last non-empty one contribute only their first empty cell); and, for the
+// corner lower bound, ediv[d-1] = ceil(n_sel / d) for d = 1..k.  One warp.
+__device__ inline void build_staircase(int k, int n_sel, uint32_t* stair, uint32_t* front,
+                                       int* ediv) {
   const int lane = threadIdx.x & 31;
+  for (int d = lane + 1; d <= k; d += 32) ediv[d - 1] = (n_sel + d - 1) / d;  // ceil(n_sel / d)
   int obase = 0, fbase = 0, prev_last = -1;
   for (int a0 = 0; a0 < k; a0 += 32) {
     const int a = a0 + lane;

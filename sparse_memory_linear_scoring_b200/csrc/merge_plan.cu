@@ -66,13 +66,15 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   uint32_t* frontW = stairW + p.ncW;
   uint32_t* stairR = frontW + p.nfW;
   uint32_t* frontR = stairR + p.ncR;
+  int* edivW = reinterpret_cast<int*>(frontR + p.nfR);
+  int* edivR = edivW + p.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int bh = blockIdx.y;
   const int s0 = blockIdx.x * kMergeSteps;
   if (s0 >= tlen) return;
   const int np = min(kMergeSteps, tlen - s0);
-  if (warp == 0) build_staircase(p.k, p.W, stairW, frontW);
-  if (warp == 1) build_staircase(p.k, p.R, stairR, frontR);
+  if (warp == 0) build_staircase(p.k, p.W, stairW, frontW, edivW);
+  if (warp == 1) build_staircase(p.k, p.R, stairR, frontR, edivR);
   __syncthreads();
   unsigned char* mine = smem + L.uni + L.per_warp * warp;
   uint64_t* h1 = reinterpret_cast<uint64_t*>(mine);
@@ -90,7 +92,8 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     uint32_t* s_out = reinterpret_cast<uint32_t*>(side ? io.out_ir : io.out_iw) + row * n_sel;
     merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
               io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
-              side ? frontR : frontW, side ? p.nfR : p.nfW, h1, h2, cand, cell, alt, sel,
+              side ? frontR : frontW, side ? p.nfR : p.nfW, side ? edivR : edivW, h1, h2, cand,
+              cell, alt, sel,
               io.sorted != 0, w_out, s_out, st, int(hr), p.rule == 1 && side == 0);
   }
 }

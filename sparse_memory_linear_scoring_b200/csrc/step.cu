@@ -137,8 +137,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) k_step(Plan p, StepIO io) {
   uint32_t* frontW = stairW + p.ncW;
   uint32_t* stairR = frontW + p.nfW;
   uint32_t* frontR = stairR + p.ncR;
-  if (warp == 0) build_staircase(k, p.W, stairW, frontW);
-  if (warp == 1) build_staircase(k, p.R, stairR, frontR);
+  int* edivW = reinterpret_cast<int*>(frontR + p.nfR);
+  int* edivR = edivW + p.k;
+  if (warp == 0) build_staircase(k, p.W, stairW, frontW, edivW);
+  if (warp == 1) build_staircase(k, p.R, stairR, frontR, edivR);
   if (tid == 0) {
     st->flags = 0;
     st->info = -1;
@@ -153,35 +155,51 @@ __global__ void __launch_bounds__(kStepThreads, 1) k_step(Plan p, StepIO io) {
     }
     __syncthreads();
     // ---- 2. scores of both halves, both sides: RPW codebook rows per warp
-    // iteration, LPRW lanes per row, EPL elements per lane
+    // load, LPRW lanes per row, EPL elements per lane; kUnr loads in flight
+    // per warp before their products; each codebook row serves k' and q'
     {
+      constexpr int kUnr = 4;
       const int sub = lane / LPRW, part = lane % LPRW;
-      for (int r0 = warp * RPW; r0 < 2 * n; r0 += kStepWarps * RPW) {
-        const int r = r0 + sub;
-        const bool ok = r < 2 * n;
-        const int half = ok && r >= n ? 1 : 0;
-        const int j = ok ? r - half * n : 0;
-        float pk = 0.f, pq = 0.f;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float xk[EPL], xq[EPL];
 #pragma unroll
-        for (int c = part * EPL; c < dh; c += LPRW * EPL) {
-          float cb[EPL];
-          ld16<Tin>((half ? c2 : c1) + size_t(j) * dh + c, cb);
-          const float* xk = xs + half * dh + c;
-          const float* xq = xs + dqk + half * dh + c;
+        for (int e = 0; e < EPL; ++e) {
+          xk[e] = xs[half * dh + part * EPL + e];
+          xq[e] = xs[dqk + half * dh + part * EPL + e];
+        }
+        const Tin* cbh = (half ? c2 : c1) + part * EPL;
+        for (int j0 = warp * RPW * kUnr; j0 < n; j0 += kStepWarps * RPW * kUnr) {
+          float cb[kUnr][EPL];
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            pk = fmaf(xk[e], cb[e], pk);
-            pq = fmaf(xq[e], cb[e], pq);
+          for (int u = 0; u < kUnr; ++u) {
+            const int j = j0 + u * RPW + sub;
+            if (j < n) {
+              ld16<Tin>(cbh + size_t(j) * dh, cb[u]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) cb[u][e] = 0.f;
+            }
           }
-        }
 #pragma unroll
-        for (int off = LPRW / 2; off > 0; off >>= 1) {
-          pk += __shfl_xor_sync(0xffffffffu, pk, off);
-          pq += __shfl_xor_sync(0xffffffffu, pq, off);
-        }
-        if (ok && part == 0) {
-          sc[(0 * 2 + half) * n + j] = pk;
-          sc[(1 * 2 + half) * n + j] = pq;
+          for (int u = 0; u < kUnr; ++u) {
+            float pk = 0.f, pq = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              pk = fmaf(xk[e], cb[u][e], pk);
+              pq = fmaf(xq[e], cb[u][e], pq);
+            }
+#pragma unroll
+            for (int off = LPRW / 2; off > 0; off >>= 1) {
+              pk += __shfl_xor_sync(0xffffffffu, pk, off);
+              pq += __shfl_xor_sync(0xffffffffu, pq, off);
+            }
+            const int j = j0 + u * RPW + sub;
+            if (j < n && part == 0) {
+              sc[(0 * 2 + half) * n + j] = pk;
+              sc[(1 * 2 + half) * n + j] = pq;
+            }
+          }
         }
       }
     }
@@ -222,7 +240,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) k_step(Plan p, StepIO io) {
       uint32_t* s_out = sels + (side ? p.W : 0);
       merge_one(p, hl + size_t(side * 2) * K2, k, hl + size_t(side * 2 + 1) * K2, k, n_sel,
                 side ? stairR : stairW, side ? p.ncR : p.ncW, side ? frontR : frontW,
-                side ? p.nfR : p.nfW, h1, h2, cand, cell, alt, sel, lists, w_out, s_out, st, t);
+                side ? p.nfR : p.nfW, side ? edivR : edivW, h1, h2, cand, cell, alt, sel, lists,
+                w_out, s_out, st, t);
       if (lists) {
         int32_t* gi = (side ? io.idx_r : io.idx_w) + row * n_sel;
         float* gw = (side ? io.w_r : io.w_w) + row * n_sel;
