@@ -249,6 +249,37 @@ SDM_API int sdm_get_device_status(const void* workspace, size_t ws_bytes, int32_
 SDM_API const char* sdm_status_string(int status);
 
 /*
+ * Gradients of the forward pass, for training (the pages make the initial
+ * table M_0 a learned parameter, "Estado Inicial Aprendido"; they give no
+ * backward pass).  The gradient is that of "Mecanismo Central" items 2-4 with
+ * the discrete choices (each half's top-k, the top-W / top-R candidates) held
+ * at the ones the forward made -- they are piecewise constant in the inputs.
+ * Given the forward's inputs, the table it started from (M0, read only: keep a
+ * copy, since sdm_forward overwrites M_inout), its selections as sdm_select
+ * writes them (idx_w, w_w, idx_r, w_r; any order within a step), d_o = dL/do
+ * [B][H][T][d_v] float32 and dM_T = dL/dM_T [B][H][N][d_v] float32 (NULL for
+ * 0), it writes float32 dq, dk [B][H][T][d_qk], dv [B][H][T][d_v], dalpha,
+ * dbeta [B][H][T], dC1, dC2 [H][n_sub][d_qk/2] and dM0 [B][H][N][d_v].
+ * The whole sequence is one call (a long sequence is split by the caller:
+ * segments backward in reverse order, each given the table at its start and
+ * the dM0 of the segment after it as its dM_T); the workspace
+ * (sdm_backward_workspace_bytes) holds the plan and the row each access of the
+ * forward saw, (2W + R) d_v floats per token-head, plus a working copy of M0.
+ * The codebook gradients are accumulated with float atomics, so their last
+ * bits vary from call to call.  Same pointer, stream and error conventions as
+ * sdm_forward (dalpha, dbeta: 4-byte alignment).
+ */
+SDM_API size_t sdm_backward_workspace_bytes(const sdm_dims* dims);
+
+SDM_API int sdm_backward(const void* q, const void* k, const void* v, const float* alpha,
+                         const float* beta, const void* C1, const void* C2, const float* M0,
+                         const int32_t* idx_w, const float* w_w, const int32_t* idx_r,
+                         const float* w_r, const float* d_o, const float* dM_T, float* dq,
+                         float* dk, float* dv, float* dalpha, float* dbeta, float* dC1,
+                         float* dC2, float* dM0, const sdm_dims* dims, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/*
  * Dense Gated DeltaNet (GDN) baseline, for comparison at matched sizes (the
  * SDM summaries' "Resultados": SDM trains 1.49x slower than the dense GDN, an
  * HBM-against-SRAM difference).  Per (b,h) head a dense state S in

@@ -47,25 +47,33 @@ def forward64(x: Dict[str, torch.Tensor], lists: Dict[str, np.ndarray], dims: Di
     for b in range(B):
         ob, Mb = [], []
         for h in range(H):
-            M = x['M0'][b, h]
+            # only the rows the head ever selects take part: a compact table of
+            # them (gathered from M0, so its gradient flows back to M0)
+            iw = lists['idx_w'][b, h].astype(np.int64)
+            ir = lists['idx_r'][b, h].astype(np.int64)
+            rows = np.unique(np.concatenate([iw.reshape(-1), ir.reshape(-1)]))
+            rows_t = torch.as_tensor(rows)
+            M = x['M0'][b, h][rows_t]
             C1, C2 = x['C1'][h], x['C2'][h]
             oh = []
             for t in range(T):
                 kt, qt = x['k'][b, h, t], x['q'][b, h, t]
-                ws = torch.as_tensor(lists['idx_w'][b, h, t].astype(np.int64))
-                rs = torch.as_tensor(lists['idx_r'][b, h, t].astype(np.int64))
+                ws = torch.as_tensor(iw[t])
+                rs = torch.as_tensor(ir[t])
+                cw = torch.as_tensor(np.searchsorted(rows, iw[t]))
+                cr = torch.as_tensor(np.searchsorted(rows, ir[t]))
                 sw = (C1[ws // n] @ kt[:dh]) + (C2[ws % n] @ kt[dh:])
                 sr = (C1[rs // n] @ qt[:dh]) + (C2[rs % n] @ qt[dh:])
                 w = torch.softmax(sw, 0)
                 u = torch.softmax(sr, 0)
                 c = x['beta'][b, h, t] * w
-                Mt = x['alpha'][b, h, t] * M[ws]
+                Mt = x['alpha'][b, h, t] * M[cw]
                 new = (1.0 - c)[:, None] * Mt + c[:, None] * x['v'][b, h, t][None, :]
-                M = M.index_copy(0, ws, new)
-                oh.append(u @ M[rs])
+                M = M.index_copy(0, cw, new)
+                oh.append(u @ M[cr])
             ob.append(torch.stack(oh) if oh else torch.zeros(0, x['v'].shape[-1],
                                                              dtype=torch.float64))
-            Mb.append(M)
+            Mb.append(x['M0'][b, h].index_copy(0, rows_t, M))
         os_.append(torch.stack(ob))
         Ms.append(torch.stack(Mb))
     return torch.stack(os_), torch.stack(Ms)

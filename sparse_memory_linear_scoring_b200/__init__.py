@@ -8,6 +8,6 @@ without the built library, or with CPU tensors, raises.
 """
 from .sdm import (  # noqa: F401
     SDMError, Dims, LIB_PATH, load_library, workspace_bytes, forward, forward_decay, step, select,
-    recur,
+    recur, backward,
     device_status, make_dims, query_plan, PLAN_FIELDS, gdn_forward, gdn_workspace_bytes, GdnDims,
 )

@@ -260,12 +260,15 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
         r.w = __float_as_int(c);
       }
       rec[b0 + rank] = r;
+      if (io.rent) io.rent[(size_t(bh) * p.nblk + blk) * p.E + b0 + rank] = e;
     }
   }
   // the recurrence adds every read into o with reductions: start from zero
-  float4* o4 = reinterpret_cast<float4*>(io.o + trow0 * p.dv);
-  const int n4 = np * p.dv / 4;
-  for (int i = tid; i < n4; i += stride) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (io.o) {
+    float4* o4 = reinterpret_cast<float4*>(io.o + trow0 * p.dv);
+    const int n4 = np * p.dv / 4;
+    for (int i = tid; i < n4; i += stride) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 cudaError_t launch_merge(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,

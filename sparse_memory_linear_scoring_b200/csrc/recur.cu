@@ -171,7 +171,7 @@ __device__ __forceinline__ void cp_bytes(void* dst, const void* src) {
 }
 
 #ifndef SDM_RECUR_VREG
-#define SDM_RECUR_VREG 0
+#define SDM_RECUR_VREG 1
 #endif
 
 template <typename Tv, int LPR, int F>
@@ -191,11 +191,11 @@ struct RecurSmem {
   static constexpr size_t total = per_stream * kStreams;
 };
 
-template <typename Tv, int LPR, int F>
+template <typename Tv, int LPR, int F, bool SAVE>
 __global__ void __launch_bounds__(kRecurThreads, kRecurWarps / 148 / (kRecurThreads / 32))
 k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restrict__ o,
         const int4* __restrict__ rec, const int* __restrict__ roff, int t0, int tlen, int bh0,
-        int nbh) {
+        int nbh, float* __restrict__ snap) {
   using SM = RecurSmem<Tv, LPR, F>;
   constexpr int dv = LPR * F;
   constexpr int U = SM::U;
@@ -359,6 +359,12 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
 #pragma unroll
           for (int j = 0; j < F; ++j) cur[j] = mrow[u * dv + j];
         }
+        if constexpr (SAVE) {
+          // the row as this record finds it (record index as in rec)
+          const size_t ri = u < t1 ? (size_t(bh) * p.nblk + b) * p.E + pos + u
+                                   : (size_t(bh) * p.nblk + b + 1) * p.E + npos + (u - t1);
+          st_row<F>(snap + ri * dv + sl * F, cur);
+        }
         if (!(r.y & 1)) {
 #pragma unroll
           for (int j = 0; j < F; ++j) {
@@ -368,7 +374,7 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
             cur[j] = fmaf(f1, cur[j], f2 * vj);
           }
           dirty = true;
-        } else {
+        } else if constexpr (!SAVE) {
           red_row<F>(oh + size_t(r.y >> 1) * dv, cur, f1);
         }
         if ((last >> u) & 1u) {
@@ -400,12 +406,12 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
   cp_async_wait_all();
 }
 
-template <typename Tv, int LPR, int F>
+template <typename Tv, int LPR, int F, bool SAVE>
 static cudaError_t launch_recur_t(const Plan& p, const void* v, float* M, float* o,
                                   const int4* rec, const int* roff, int t0, int tlen,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, float* snap) {
   const size_t smem = RecurSmem<Tv, LPR, F>::total;
-  cudaError_t e = cudaFuncSetAttribute(k_recur<Tv, LPR, F>,
+  cudaError_t e = cudaFuncSetAttribute(k_recur<Tv, LPR, F, SAVE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   // heads in groups of p.HG per launch, so that the rows in use at a time
@@ -414,8 +420,8 @@ static cudaError_t launch_recur_t(const Plan& p, const void* v, float* M, float*
     const int nbh = min(p.HG, p.BH - bh0);
     const long long threads = (long long)nbh * p.S * LPR;
     const int grid = int((threads + kRecurThreads - 1) / kRecurThreads);
-    k_recur<Tv, LPR, F><<<grid, kRecurThreads, smem, s>>>(p, (const Tv*)v, M, o, rec, roff, t0,
-                                                          tlen, bh0, nbh);
+    k_recur<Tv, LPR, F, SAVE><<<grid, kRecurThreads, smem, s>>>(
+        p, (const Tv*)v, M, o, rec, roff, t0, tlen, bh0, nbh, snap);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -434,31 +440,32 @@ int recur_lanes_per_row(int dv) { return dv / recur_floats_per_lane(dv); }
 template <typename Tv, int DV>
 static cudaError_t launch_recur_w(const Plan& p, const void* v, float* M, float* o,
                                   const int4* rec, const int* roff, int t0, int tlen,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, float* snap) {
   constexpr int F = recur_floats_per_lane(DV);
-  return launch_recur_t<Tv, DV / F, F>(p, v, M, o, rec, roff, t0, tlen, s);
+  if (snap) return launch_recur_t<Tv, DV / F, F, true>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+  return launch_recur_t<Tv, DV / F, F, false>(p, v, M, o, rec, roff, t0, tlen, s, nullptr);
 }
 
 template <typename Tv>
 static cudaError_t launch_recur_dt(const Plan& p, const void* v, float* M, float* o,
                                    const int4* rec, const int* roff, int t0, int tlen,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, float* snap) {
   switch (p.dv) {
-    case 4: return launch_recur_w<Tv, 4>(p, v, M, o, rec, roff, t0, tlen, s);
-    case 8: return launch_recur_w<Tv, 8>(p, v, M, o, rec, roff, t0, tlen, s);
-    case 16: return launch_recur_w<Tv, 16>(p, v, M, o, rec, roff, t0, tlen, s);
-    case 32: return launch_recur_w<Tv, 32>(p, v, M, o, rec, roff, t0, tlen, s);
-    case 64: return launch_recur_w<Tv, 64>(p, v, M, o, rec, roff, t0, tlen, s);
-    case 128: return launch_recur_w<Tv, 128>(p, v, M, o, rec, roff, t0, tlen, s);
+    case 4: return launch_recur_w<Tv, 4>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    case 8: return launch_recur_w<Tv, 8>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    case 16: return launch_recur_w<Tv, 16>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    case 32: return launch_recur_w<Tv, 32>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    case 64: return launch_recur_w<Tv, 64>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    case 128: return launch_recur_w<Tv, 128>(p, v, M, o, rec, roff, t0, tlen, s, snap);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_recur(const Plan& p, const void* v, float* M, float* o, const int4* rec,
-                         const int* roff, int t0, int tlen, cudaStream_t s) {
+                         const int* roff, int t0, int tlen, cudaStream_t s, float* snap) {
   if (p.dtype == SDM_DTYPE_F32)
-    return launch_recur_dt<float>(p, v, M, o, rec, roff, t0, tlen, s);
-  return launch_recur_dt<__nv_bfloat16>(p, v, M, o, rec, roff, t0, tlen, s);
+    return launch_recur_dt<float>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+  return launch_recur_dt<__nv_bfloat16>(p, v, M, o, rec, roff, t0, tlen, s, snap);
 }
 
 }  // namespace sdm

@@ -200,11 +200,17 @@ struct PlanIO {
   int4* rec;
   int* roff;
   float* o;
+  int* rent;  // optional: the block-local list entry (step * (W + R) + j) of each record
 };
 cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevStatus* st,
                         cudaStream_t s);
 
+// snap == nullptr: the recurrence (writes into M, reads added into o).  snap
+// given: the same walk over M, with no o, storing at every record the row it
+// sees before the record's effect (snap[record] = d_v floats, record index as
+// in rec) -- the values the backward pass needs.
 cudaError_t launch_recur(const Plan& p, const void* v, float* M, float* o, const int4* rec,
-                         const int* roff, int t0, int tlen, cudaStream_t s);
+                         const int* roff, int t0, int tlen, cudaStream_t s,
+                         float* snap = nullptr);
 
 }  // namespace sdm

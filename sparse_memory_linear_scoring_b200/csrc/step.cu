@@ -6,9 +6,10 @@
 // step t (the same method as sdm_forward):
 //   1. scoring (item 2): the two halves of k'_t and q'_t against C1 and C2, on
 //      CUDA cores (float32 FMA), into shared memory: 4 x n scores;
-//   2. per-half top-k (item 2): one warp per (side, half) finds the k-th
-//      largest score by a bitwise search over order-preserving images and
-//      sorts the k best by (score desc, row asc);
+//   2. per-half top-k (item 2): four warps per (side, half) find the k-th
+//      largest score by a bitwise search over order-preserving images (their
+//      counts added through shared memory), and the k best are sorted by
+//      (score desc, row asc);
 //   3. merge (item 2): one warp per side takes the top-W (k') / top-R (q') of
 //      the k x k outer-sum candidates with the staircase merge of sdm_forward,
 //      and their softmax weights;
@@ -31,7 +32,7 @@ constexpr int kStepMaxN = 1024;   // scores of a half-row held 32 per lane
 constexpr int kStepMaxK = 256;
 
 struct StepLayout {
-  size_t x, sc, tk, hl, merge, selw, sels, opart, st, total;
+  size_t x, sc, tk, hl, merge, selw, sels, opart, st, xch, total;
   int K2;
   MergeLayout ML;
 };
@@ -50,6 +51,8 @@ __host__ __device__ inline StepLayout step_layout(const Plan& p) {
   L.sels = o; o = al16(o + size_t(p.W + p.R) * 4);       // slots: write, then read
   L.opart = o; o = al16(o + size_t(kStepWarps) * p.dv * 4);
   L.st = o; o = al16(o + sizeof(DevStatus));
+  L.xch = o; o = al16(o + size_t(4) * 8 * 4);              // top-k count exchange
+
   L.total = o;
   return L;
 }
@@ -97,6 +100,101 @@ __device__ __forceinline__ float4 ld_v4<__nv_bfloat16>(const __nv_bfloat16* ptr)
                      __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
 }
 
+// The k best of one half-row's n <= 1024 scores (sc), found by the four warps of
+// a group: warp `part` holds entries [256 part, 256 part + 256), 8 per lane,
+// in row order.  The k-th largest order-preserving image comes from a bitwise
+// search whose per-bit counts the four warps add through shared memory (xch,
+// [2][4] ints, double-buffered by bit parity) behind the group's named barrier
+// `bar` (128 threads); the k best -- ties at the threshold to the lowest rows,
+// i.e. in warp then lane order -- are written to out[0..k) as 64-bit keys.
+__device__ __forceinline__ void group_bar(int bar) {
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+}
+
+__device__ void group_topk(const float* sc, int n, int k, int part, int bar, int* xch,
+                           uint64_t* out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[8];
+  uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int j = part * 256 + u * 32 + lane;
+    key[u] = j < n ? f2ord(sc[j]) : 0u;  // 0: below every valid image
+    if (j < n) {
+      lo = min(lo, key[u]);
+      hi = max(hi, key[u]);
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    xch[part] = int(lo);
+    xch[4 + part] = int(hi);
+  }
+  group_bar(bar);
+  lo = min(min(uint32_t(xch[0]), uint32_t(xch[1])), min(uint32_t(xch[2]), uint32_t(xch[3])));
+  hi = max(max(uint32_t(xch[4]), uint32_t(xch[5])), max(uint32_t(xch[6]), uint32_t(xch[7])));
+  group_bar(bar);  // everyone has read lo/hi before the slots are reused
+  uint32_t thr = hi;
+  const uint32_t diff = lo ^ hi;
+  if (diff != 0u) {
+    const int top = 31 - __clz(diff);
+    thr = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t cand = thr | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) c += key[u] >= cand ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      int* slot = xch + (bit & 1) * 4;
+      if (lane == 0) slot[part] = c;
+      group_bar(bar);
+      if (slot[0] + slot[1] + slot[2] + slot[3] >= k) thr = cand;
+    }
+  }
+  // the entries above thr, then the lowest rows equal to it
+  int ngt = 0, neq = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    ngt += key[u] > thr ? 1 : 0;
+    neq += (key[u] == thr && part * 256 + u * 32 + lane < n) ? 1 : 0;
+  }
+  ngt = __reduce_add_sync(0xffffffffu, ngt);
+  neq = __reduce_add_sync(0xffffffffu, neq);
+  group_bar(bar);  // the last bit's counts have been read
+  if (lane == 0) {
+    xch[part] = ngt;
+    xch[4 + part] = neq;
+  }
+  group_bar(bar);
+  int gt_all = 0, eq_before = 0, gt_before = 0;
+  for (int w = 0; w < 4; ++w) {
+    gt_all += xch[w];
+    if (w < part) {
+      eq_before += xch[4 + w];
+      gt_before += xch[w];
+    }
+  }
+  const int m = k - gt_all;  // ties to take overall, lowest rows first
+  int ties_here = min(max(m - eq_before, 0), neq);
+  int eq_taken_before = min(max(m, 0), eq_before);
+  int base = gt_before + eq_taken_before;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int j = part * 256 + u * 32 + lane;
+    const bool above = key[u] > thr;
+    const bool tie = key[u] == thr && j < n;
+    const unsigned mt = __ballot_sync(0xffffffffu, tie);
+    const int trank = __popc(mt & lt);
+    const bool take = above || (tie && trank < ties_here);
+    const unsigned mk = __ballot_sync(0xffffffffu, take);
+    if (take) out[base + __popc(mk & lt)] = (uint64_t(key[u]) << 32) | uint64_t(~uint32_t(j));
+    base += __popc(mk);
+    ties_here -= min(ties_here, __popc(mt));
+  }
+}
+
 struct StepIO {
   const void *q, *k, *v;
   const float *alpha, *beta;
@@ -118,6 +216,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) k_step(Plan p, StepIO io) {
   uint32_t* sels = reinterpret_cast<uint32_t*>(smem + L.sels);
   float* opart = reinterpret_cast<float*>(smem + L.opart);
   DevStatus* st = reinterpret_cast<DevStatus*>(smem + L.st);
+  int* xch = reinterpret_cast<int*>(smem + L.xch);
   constexpr int EPL = step_epl<Tin>();
   constexpr int RPW = 32 / LPRW;  // codebook rows per warp and iteration
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -204,25 +303,20 @@ __global__ void __launch_bounds__(kStepThreads, 1) k_step(Plan p, StepIO io) {
       }
     }
     __syncthreads();
-    // ---- 3. exact sorted top-k of each of the four half-rows
-    if (warp < 4) {
-      uint32_t key[32], rw[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int j = i * 32 + lane;
-        key[i] = j < n ? f2ord(sc[warp * n + j]) : 0u;
-        rw[i] = uint32_t(j);
+    // ---- 3. exact sorted top-k of each of the four half-rows, four warps each
+    {
+      const int hrw = warp >> 2, part = warp & 3;
+      uint64_t* out = tk + size_t(hrw) * K2;
+      group_topk(sc + size_t(hrw) * n, n, k, part, 1 + hrw, xch + hrw * 8, out);
+      group_bar(1 + hrw);
+      if (part == 0) {
+        for (int i = k + lane; i < K2; i += 32) out[i] = 0;
+        __syncwarp();
+        warp_sort_desc(out, K2);
+        uint2* hw = hl + size_t(hrw) * K2;
+        for (int i = lane; i < k; i += 32)
+          hw[i] = make_uint2(__float_as_uint(key_val(out[i])), key_idx(out[i]));
       }
-      uint64_t* out = tk + size_t(warp) * K2;
-      const uint32_t thr = warp_kth_key<32>(key, n, k);
-      warp_gather_topk<32>(key, rw, n, k, thr, out);
-      __syncwarp();
-      for (int i = k + lane; i < K2; i += 32) out[i] = 0;
-      __syncwarp();
-      warp_sort_desc(out, K2);
-      uint2* hw = hl + size_t(warp) * K2;
-      for (int i = lane; i < k; i += 32)
-        hw[i] = make_uint2(__float_as_uint(key_val(out[i])), key_idx(out[i]));
     }
     __syncthreads();
     // ---- 4. merge: warp 0 the write slots (k'), warp 1 the read slots (q')

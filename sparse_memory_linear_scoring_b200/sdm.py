@@ -72,6 +72,10 @@ def load_library():
             lib.sdm_gdn_forward.restype = ctypes.c_int
             lib.sdm_forward_decay.argtypes = [P] * 8 + [DP, P, S, P]
             lib.sdm_forward_decay.restype = ctypes.c_int
+            lib.sdm_backward_workspace_bytes.argtypes = [DP]
+            lib.sdm_backward_workspace_bytes.restype = S
+            lib.sdm_backward.argtypes = [P] * 22 + [DP, P, S, P]
+            lib.sdm_backward.restype = ctypes.c_int
             lib.sdm_step.argtypes = [P] * 13 + [DP, P]
             lib.sdm_step.restype = ctypes.c_int
             lib.sdm_version.argtypes = []
@@ -296,6 +300,49 @@ def step(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
                                    _ptr(C2), _ptr(M), _ptr(o), *[_ptr(x) for x in lw],
                                    ctypes.byref(dims), _stream(dev, stream)))
     return (o, *lw) if lists else o
+
+
+def backward(q, k, v, alpha, beta, C1, C2, M0, idx_w, w_w, idx_r, w_r, d_o, dM_T=None, *,
+             topk: int, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of the forward pass at its selections (sdm_backward).  M0 is the
+    table the forward started from; the lists are sdm_select's; d_o = dL/do,
+    dM_T = dL/dM_T (None: 0).  Returns a dict of float32 gradients: q, k, v,
+    alpha, beta, C1, C2, M0."""
+    B, H, T, d_qk, n_sub, dt = _check_inputs(q, k, v, C1, C2, alpha, beta)
+    d_v = v.shape[-1]
+    W, R = idx_w.shape[-1], idx_r.shape[-1]
+    N = n_sub * n_sub
+    _expect(M0, "M0", (B, H, N, d_v), (torch.float32,))
+    _expect(idx_w, "idx_w", (B, H, T, W), (torch.int32,))
+    _expect(w_w, "w_w", (B, H, T, W), (torch.float32,))
+    _expect(idx_r, "idx_r", (B, H, T, R), (torch.int32,))
+    _expect(w_r, "w_r", (B, H, T, R), (torch.float32,))
+    _expect(d_o, "d_o", (B, H, T, d_v), (torch.float32,))
+    if dM_T is not None:
+        _expect(dM_T, "dM_T", (B, H, N, d_v), (torch.float32,))
+    dev = _dev(q, k, v, alpha, beta, C1, C2, M0, idx_w, w_w, idx_r, w_r, d_o,
+               *([dM_T] if dM_T is not None else []))
+    dims = make_dims(B, H, T, d_qk, d_v, n_sub, topk, W, R, dt)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = dict(q=torch.empty(B, H, T, d_qk, **f32), k=torch.empty(B, H, T, d_qk, **f32),
+             v=torch.empty(B, H, T, d_v, **f32), alpha=torch.empty(B, H, T, **f32),
+             beta=torch.empty(B, H, T, **f32), C1=torch.empty(H, n_sub, d_qk // 2, **f32),
+             C2=torch.empty(H, n_sub, d_qk // 2, **f32), M0=torch.empty(B, H, N, d_v, **f32))
+    lib = load_library()
+    need = int(lib.sdm_backward_workspace_bytes(ctypes.byref(dims)))
+    if need == 0:
+        _check(lib.sdm_backward(*([None] * 22), ctypes.byref(dims), None, 0, None))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or _nbytes(workspace) < need or not workspace.is_contiguous():
+        raise SDMError(4, "workspace too small, not contiguous or on another device")
+    _check(lib.sdm_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(C1),
+                            _ptr(C2), _ptr(M0), _ptr(idx_w), _ptr(w_w), _ptr(idx_r), _ptr(w_r),
+                            _ptr(d_o), _ptr(dM_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
+                            _ptr(g["alpha"]), _ptr(g["beta"]), _ptr(g["C1"]), _ptr(g["C2"]),
+                            _ptr(g["M0"]), ctypes.byref(dims), _ptr(workspace),
+                            _nbytes(workspace), _stream(dev, stream)))
+    return g
 
 
 def gdn_forward(q, k, v, alpha, beta, S, *, o: Optional[torch.Tensor] = None,
