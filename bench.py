@@ -634,10 +634,14 @@ def decode(cfg, steps):
         return {"eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
                 "graph_token_heads_per_s": cfg.BH / (graph_us * 1e-6)}
 
+    clocks = ClockSampler(_device_uuid(torch, torch.device("cuda")))
+    clocks.start()
     res = {"sdm_step": timed(one_step), "sdm_forward_T1": timed(one_forward)}
+    clk = clocks.stop()
     st, info = sdm.device_status(ws)
     return {"decode": "one call per step, M carried", "workload": workload_desc(cfg),
-            "steps": steps, "heads": cfg.BH, "kernels": res, "device_status": st}
+            "steps": steps, "heads": cfg.BH, "kernels": res, "device_status": st,
+            "clocks": clk}
 
 
 def gdn_compare(cfg, steps, warmup):
@@ -677,10 +681,13 @@ def gdn_compare(cfg, steps, warmup):
             tot += e0.elapsed_time(e1)
         return tot / steps
 
+    clocks = ClockSampler(_device_uuid(torch, torch.device("cuda")))
+    clocks.start()
     gdn_ms = time_it(lambda: sdm.gdn_forward(g["q"], g["k"], g["v"], g["alpha"], g["beta"], S,
                                              o=og, workspace=ws))
     sdm_ms = time_it(lambda: sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"],
                                          d["C2"], M, topk=cfg.k, W=cfg.W, R=cfg.R, o=osd))
+    clk = clocks.stop()
     th = cfg.BH * cfg.T
     return {"baseline": "dense Gated DeltaNet (sdm_gdn_forward), matched d_k = W",
             "workload": workload_desc(cfg), "gdn": {"d_k": cfg.W, "d_v": cfg.d_v,
@@ -689,7 +696,7 @@ def gdn_compare(cfg, steps, warmup):
             "sdm": {"ms_per_step": sdm_ms, "token_heads_per_s": th / (sdm_ms / 1e3)},
             "sdm_over_gdn_time": sdm_ms / gdn_ms,
             "pages": "SDM trains 1.49x slower than GDN at 8B (other hardware, training)",
-            "steps": steps, "l2": "flushed before each step"}
+            "steps": steps, "l2": "flushed before each step", "clocks": clk}
 
 
 def main():

@@ -15,10 +15,11 @@
 //   warps 2..17 epilogue, kQ = 4 threads per token row (the kQ warps whose
 //               warp index is equal mod 4 share one 32-lane TMEM quarter; each
 //               takes a quarter of every 256-column tile): tcgen05.ld the
-//               row's scores, keep those above a threshold tau taken from the
-//               row's own score mean and deviation (first 512 columns), then
-//               select the exact top-k of the kept scores and write them sorted
-//               by (score desc, row asc).
+//               row's scores and keep those above a threshold tau taken from
+//               the row's own score mean and deviation (first 512 columns);
+//               then, one warp per row, the exact top-k of the kept scores
+//               (bitwise search of the k-th, gather, warp sort), written
+//               sorted by (score desc, row asc).
 // A row whose kept count falls outside [k, capacity] (or whose scores do not
 // spread) is queued for the exact CUDA-core path instead, so the result is
 // exact for any input.  Every mbarrier wait is bounded: on a timeout the CTA
@@ -31,7 +32,7 @@
 
 #include <mutex>
 
-#include "sdm_internal.cuh"
+#include "select_dev.cuh"
 
 namespace sdm {
 namespace {
@@ -42,7 +43,6 @@ constexpr int kKAtom = 64;           // bf16 elements per 128-byte swizzle row
 constexpr int kQ = 4;                // epilogue threads per token row
 constexpr int kEpiThreads = kQ * kTileM;
 constexpr int kThreads = 64 + kEpiThreads;
-constexpr int kBuckets = 64;         // final-selection buckets per row
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 constexpr uint32_t kATileBytes = kTileM * 128;   // one 64-column chunk of the token tile
 constexpr uint32_t kBTileBytes = kTileN * 128;   // one 64-column chunk of a codebook tile
@@ -57,8 +57,12 @@ struct TcArgs {
   DevStatus* st;
 };
 
+// Per-row survivor lists are row-major with one element of padding (row
+// stride C + 1 floats, C + 2 row numbers), so that the filter's appends (one
+// lane per row) and the selection's reads (one warp per row) both spread over
+// the banks.
 struct TcLayout {
-  uint32_t a, b, vals, idx, hist, rows, bars, total;
+  uint32_t a, b, vals, idx, rows, bars, total;
   int nkc;
 };
 
@@ -68,21 +72,20 @@ __host__ __device__ inline TcLayout tc_layout(const Plan& p) {
   uint32_t o = 0;
   L.a = o; o += L.nkc * kATileBytes;
   L.b = o; o += 2 * L.nkc * kBTileBytes;
-  L.vals = o; o += uint32_t(p.C) * kTileM * 4;
-  L.idx = o; o += uint32_t(p.C) * kTileM * 2;
+  L.vals = o; o += uint32_t(p.C + 1) * kTileM * 4;
+  L.idx = o; o += uint32_t(p.C + 2) * kTileM * 2;
   o = (o + 15) & ~15u;
-  L.hist = o; o += (kBuckets / 4) * kTileM * 4;
-  L.rows = o; o += (2 + 4 * kQ) * kTileM * 4;  // per-row count, nout, partial stats
+  L.rows = o; o += (2 + 2 * kQ) * kTileM * 4;  // per-row count, go flag, partial stats
   o = (o + 15) & ~15u;
   L.bars = o; o += 16 * 8;  // mbarriers, TMEM address, abort flags
   L.total = o + 1024;  // slack for 1024-byte alignment of the dynamic base
   return L;
 }
 
-// Entries per row of the sorted-output staging area, which reuses the token
-// tile and codebook ring once every MMA has completed.
-__host__ __device__ inline int out_capacity(const TcLayout& L) {
-  return int((L.vals - L.a) / (kTileM * 8));
+// The selection's per-warp sort buffers reuse the token tile and codebook
+// ring once every MMA has completed: 16 warps x next_pow2(k) 64-bit keys.
+__host__ __device__ inline bool sort_area_fits(const TcLayout& L, int k) {
+  return uint32_t(kEpiThreads / 32) * uint32_t(next_pow2(k < 2 ? 2 : k)) * 8u <= L.vals - L.a;
 }
 
 // ---- PTX wrappers -------------------------------------------------------------
@@ -187,12 +190,8 @@ __device__ __forceinline__ void epi_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
 }
 
-// (score desc, row asc) order on the output pairs
-__device__ __forceinline__ bool before(uint2 a, uint2 b) {
-  const float va = __uint_as_float(a.x), vb = __uint_as_float(b.x);
-  return va > vb || (va == vb && a.y < b.y);
-}
 
+template <int PL>
 __global__ void __launch_bounds__(kThreads, 1)
 k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
            const __grid_constant__ CUtensorMap mc1, const __grid_constant__ CUtensorMap mc2,
@@ -205,9 +204,8 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
   const TcLayout L = tc_layout(p);
   unsigned char* sA = smem + L.a;
   unsigned char* sB = smem + L.b;
-  float* vals = reinterpret_cast<float*>(smem + L.vals);
-  uint16_t* idxs = reinterpret_cast<uint16_t*>(smem + L.idx);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);  // [16][128]
+  float* vals = reinterpret_cast<float*>(smem + L.vals);        // [128][C + 1]
+  uint16_t* idxs = reinterpret_cast<uint16_t*>(smem + L.idx);   // [128][C + 2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* full = bars;       // [2] TMA -> MMA
   uint64_t* empty = bars + 2;  // [2] MMA -> TMA
@@ -319,16 +317,11 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
     const int C = p.C;
     constexpr int kCols = kTileN / kQ;
     int* rcnt = reinterpret_cast<int*>(smem + L.rows);      // [128] kept count
-    int* rsel = rcnt + kTileM;                              // [128] nout | bstar << 16
-    float* rst = reinterpret_cast<float*>(rsel + kTileM);   // [4][kQ][128] sum, sq, min, max
-    uint32_t* h = hist + row;                               // [16][128] packed byte counts
+    int* rgo = rcnt + kTileM;                               // [128] row settled here
+    float* rst = reinterpret_cast<float*>(rgo + kTileM);    // [2][kQ][128] sum, sq
     volatile int* epi_abort = reinterpret_cast<volatile int*>(bars + 12);
     float v[32];
-    if (sub == 0) {
-      rcnt[row] = 0;
-#pragma unroll
-      for (int w = 0; w < kBuckets / 4; ++w) h[w * kTileM] = 0u;
-    }
+    if (sub == 0) rcnt[row] = 0;
     // statistics of the first (up to) two tiles
     const int nstat = ntiles < 2 ? ntiles : 2;
     float sum = 0.f, sq = 0.f;
@@ -372,7 +365,8 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       if (!valid) tau = INFINITY;
     }
     // filter: append the kept scores of this thread's columns to the row's list
-    float kmin = INFINITY, kmax = -INFINITY;
+    float* vrow = vals + row * (C + 1);
+    uint16_t* irow = idxs + row * (C + 2);
     for (int j = 0; j < ntiles && ok; ++j) {
       const int s = j & 1;
       if (j >= 2) {
@@ -393,11 +387,9 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
           for (int i = 0; i < 32; ++i) {
             if ((mask >> i) & 1u) {
               if (pos < C) {
-                vals[pos * kTileM + row] = v[i];
-                idxs[pos * kTileM + row] = uint16_t(col0 + i);
+                vrow[pos] = v[i];
+                irow[pos] = uint16_t(col0 + i);
               }
-              kmin = fminf(kmin, v[i]);
-              kmax = fmaxf(kmax, v[i]);
               ++pos;
             }
           }
@@ -407,98 +399,54 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       mbar_arrive(&tempty[s]);
     }
     if (!ok) *epi_abort = 1;
-    rst[(2 * kQ + sub) * kTileM + row] = kmin;
-    rst[(3 * kQ + sub) * kTileM + row] = kmax;
     epi_sync();
     ok = !*epi_abort;
     if (!ok && threadIdx.x == 64) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
-    // exact top-k of the kept scores, sorted: bucket by value, keep the buckets
-    // that hold the k best, rank the entries inside each bucket
-    const int cnt = rcnt[row];
     const int k = p.k;
-    const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
-    bool go = ok && valid && !redo && cnt >= k && cnt <= C;
-    // every valid row this CTA does not settle -- including all of them after a
-    // timed-out wait -- is re-scored exactly, so no later kernel reads a list
-    // this call never wrote
-    if (valid && !go && sub == 0) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
-    float vmin = INFINITY, vmax = -INFINITY;
+    if (sub == 0) {
+      const int cnt = rcnt[row];
+      const bool go = ok && valid && !redo && cnt >= k && cnt <= C;
+      rgo[row] = go ? 1 : 0;
+      // every valid row this CTA does not settle -- including all of them after
+      // a timed-out wait -- is re-scored exactly, so no later kernel reads a
+      // list this call never wrote
+      const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
+      if (valid && !go) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+    }
+    epi_sync();
+    // exact top-k of each settled row's kept scores, one warp per row: the
+    // k-th largest order-preserving image by a bitwise search, the k best
+    // gathered (ties: lowest codebook row), sorted by (score desc, row asc)
+    // and written to the survivor list.  Every MMA has completed (each thread
+    // waited for the last tile), so the token tile and codebook ring hold the
+    // warps' sort buffers.
+    const int ew = warp - 2;
+    const int K2 = next_pow2(k < 2 ? 2 : k);
+    uint64_t* sbuf = reinterpret_cast<uint64_t*>(smem + L.a) + size_t(ew) * K2;
+    for (int r = ew; r < kTileM; r += kEpiThreads / 32) {
+      if (!rgo[r]) continue;
+      const int cnt = rcnt[r];
+      const float* vr = vals + r * (C + 1);
+      const uint16_t* ir = idxs + r * (C + 2);
+      uint32_t key[PL], rw[PL];
 #pragma unroll
-    for (int j = 0; j < kQ; ++j) {
-      vmin = fminf(vmin, rst[(2 * kQ + j) * kTileM + row]);
-      vmax = fmaxf(vmax, rst[(3 * kQ + j) * kTileM + row]);
-    }
-    const float scale = vmax > vmin ? float(kBuckets) / (vmax - vmin) : 0.f;
-    auto bucket = [&](float x) { return min(kBuckets - 1, int((x - vmin) * scale)); };
-    const float* __restrict__ cv = vals + row;
-    if (go) {
-      for (int i = sub; i < cnt; i += kQ) {
-        const int b = bucket(cv[i * kTileM]);
-        atomicAdd(&h[(b >> 2) * kTileM], 1u << ((b & 3) * 8));
+      for (int i = 0; i < PL; ++i) {
+        const int jj = i * 32 + lane;
+        key[i] = jj < cnt ? f2ord(vr[jj]) : 0u;
+        rw[i] = jj < cnt ? uint32_t(ir[jj]) : 0u;
       }
-    }
-    epi_sync();
-    if (go && sub == 0) {
-      // counts never exceed the capacity (< 256), so bytes add without carry
-      int bstar = 0, cum = 0;
-      for (int w = kBuckets / 4 - 1; w >= 0 && cum < k; --w) {
-        const uint32_t c4 = h[w * kTileM];
-        for (int j = 3; j >= 0; --j) {
-          cum += (c4 >> (8 * j)) & 255u;
-          if (cum >= k) { bstar = 4 * w + j; break; }
-        }
-      }
-      // start offsets (descending bucket order) of the buckets >= bstar
-      int run = 0;
-      for (int w = kBuckets / 4 - 1; w >= (bstar >> 2); --w) {
-        const uint32_t c4 = h[w * kTileM];
-        uint32_t o4 = 0;
-        for (int j = 3; j >= 0; --j) {
-          if (4 * w + j < bstar) continue;
-          o4 |= uint32_t(run) << (8 * j);
-          run += (c4 >> (8 * j)) & 255u;
-        }
-        h[w * kTileM] = o4;
-      }
-      rsel[row] = run | (bstar << 16);
-      if (run > out_capacity(L)) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
-    }
-    epi_sync();
-    const int nout = go ? (rsel[row] & 0xffff) : 0;
-    const int bstar = go ? (rsel[row] >> 16) : 0;
-    go = go && nout <= out_capacity(L);
-    // every MMA has completed (each thread waited for the last tile), so the
-    // token tile and codebook ring are free: stage the bucketed list there
-    uint2* out = reinterpret_cast<uint2*>(smem + L.a);
-    if (go) {
-      for (int i = sub; i < cnt; i += kQ) {
-        const float x = cv[i * kTileM];
-        const int b = bucket(x);
-        if (b >= bstar) {
-          const uint32_t old = atomicAdd(&h[(b >> 2) * kTileM], 1u << ((b & 3) * 8));
-          const int pos = int((old >> ((b & 3) * 8)) & 255u);
-          out[pos * kTileM + row] = make_uint2(__float_as_uint(x), idxs[i * kTileM + row]);
-        }
-      }
-    }
-    epi_sync();
-    if (go) {
-      // h now holds each bucket's end; its start is the end of the bucket above.
-      // An entry's final rank is its bucket's start plus the entries of its own
-      // bucket that precede it; entries ranked below k go straight to the output.
+      const uint32_t thr = warp_kth_key<PL>(key, cnt, k);
+      warp_gather_topk<PL>(key, rw, cnt, k, thr, sbuf);
+      __syncwarp();
+      for (int i = k + lane; i < K2; i += 32) sbuf[i] = 0;
+      __syncwarp();
+      warp_sort_desc(sbuf, K2);
+      const size_t hr = (size_t(bh) * p.Tc + tile * kTileM + r) * 4 + side * 2 + half;
       uint2* g = a.surv + hr * C;
-      for (int i = sub; i < nout; i += kQ) {
-        const uint2 x = out[i * kTileM + row];
-        const int b = bucket(__uint_as_float(x.x));
-        const int end = int((h[(b >> 2) * kTileM] >> ((b & 3) * 8)) & 255u);
-        const int bn = b + 1;
-        const int start =
-            bn >= kBuckets ? 0 : int((h[(bn >> 2) * kTileM] >> ((bn & 3) * 8)) & 255u);
-        int rank = start;
-        for (int j = start; j < end; ++j) rank += before(out[j * kTileM + row], x) ? 1 : 0;
-        if (rank < k) g[rank] = x;
-      }
-      if (sub == 0) a.cnt[hr] = k;
+      for (int i = lane; i < k; i += 32)
+        g[i] = make_uint2(__float_as_uint(key_val(sbuf[i])), key_idx(sbuf[i]));
+      if (lane == 0) a.cnt[hr] = k;
+      __syncwarp();
     }
   }
   tc_fence_before();
@@ -838,8 +786,8 @@ int score_tc_mode(const sdm_dims* d) {
   tmp.tc = 1;
   const TcLayout L = tc_layout(tmp);
   // per-row bucket counts and offsets are packed bytes: the capacity stays below 256
-  const bool m1 = d->n_sub % kTileN == 0 && tmp.C <= 255 && L.total <= 227 * 1024 &&
-                  out_capacity(L) >= d->k + 16;
+  const bool m1 = d->n_sub % kTileN == 0 && tmp.C <= 8 * 32 && L.total <= 227 * 1024 &&
+                  sort_area_fits(L, d->k);
   tmp.tc = 2;
   tmp.C = score_tc_capacity(d, 2);
   const bool m2 = tc_layout_f(tmp).total <= 227 * 1024;
@@ -878,9 +826,22 @@ cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const v
     if (e != cudaSuccess) return e;
     k_score_tc_filter<<<grid, kThreadsF, smem, s>>>(mq, mk, mc1, mc2, a);
   } else {
-    e = cudaFuncSetAttribute(k_score_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    k_score_tc<<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+    if (p.C <= 4 * 32) {
+      e = cudaFuncSetAttribute(k_score_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(smem));
+      if (e != cudaSuccess) return e;
+      k_score_tc<4><<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+    } else if (p.C <= 5 * 32) {
+      e = cudaFuncSetAttribute(k_score_tc<5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(smem));
+      if (e != cudaSuccess) return e;
+      k_score_tc<5><<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+    } else {
+      e = cudaFuncSetAttribute(k_score_tc<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(smem));
+      if (e != cudaSuccess) return e;
+      k_score_tc<8><<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+    }
   }
   return cudaGetLastError();
 }
