@@ -78,13 +78,14 @@ __host__ __device__ inline size_t gdn_prep_smem(int dk, int dv) {
   return size_t(4) * (2 * kGdnC * (dk + 1) + kGdnC * (dv + dk) + kGdnC * (kGdnC + 1) + 2 * kGdnC);
 }
 
-template <typename Tin>
+template <typename Tin, int DK>
 __global__ void __launch_bounds__(kGdnThreads)
 k_gdn_prep(GdnPlan p, const Tin* __restrict__ q, const Tin* __restrict__ k,
            const Tin* __restrict__ v, const float* __restrict__ alpha,
            const float* __restrict__ beta, float* __restrict__ ws) {
   extern __shared__ __align__(16) float sm[];
-  const int dk = p.dk, dv = p.dv, dkp = dk + 1, Cp = kGdnC + 1, dx = dv + dk;
+  constexpr int dk = DK, dkp = DK + 1;
+  const int dv = p.dv, Cp = kGdnC + 1, dx = dv + dk;
   float* Ks = sm;
   float* Qs = Ks + kGdnC * dkp;
   float* X = Qs + kGdnC * dkp;
@@ -136,6 +137,7 @@ k_gdn_prep(GdnPlan p, const Tin* __restrict__ q, const Tin* __restrict__ k,
     float a = 0.f, pq = 0.f;
     if (j <= t && t < L) {
       float skk = 0.f, sqk = 0.f;
+#pragma unroll 16
       for (int e = 0; e < dk; ++e) {
         const float kj = Ks[j * dkp + e];
         skk = fmaf(Ks[t * dkp + e], kj, skk);
@@ -198,11 +200,12 @@ __device__ __forceinline__ void cp16(float* dst, const float* src) {
                : "memory");
 }
 
-template <int STAGES>
+template <int DK, int STAGES>
 __global__ void __launch_bounds__(kGdnThreads)
 k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float* __restrict__ o) {
   extern __shared__ __align__(16) float sm[];
-  const int dk = p.dk, dv = p.dv;
+  constexpr int dk = DK;
+  const int dv = p.dv;
   const int tid = threadIdx.x;
   const int rb = blockIdx.x, bh = blockIdx.y;
   const int i0 = rb * kGdnRB;  // first row of S
@@ -258,6 +261,7 @@ k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float
     // U[t][r] = U~[t][r] - W[t] . S[r];  o[t][r] = Q~[t] . S[r] + sum_{j<=t} P[t][j] U[j][r]
     const int lane = tid & 31, r = tid >> 6, ts = ((tid >> 5) & 1) * 32 + lane;
     float su = 0.f, sq = 0.f;
+#pragma unroll 16
     for (int e = 0; e < dk; ++e) {
       const float sv = Ss[r * dk + e];
       su = fmaf(Wt[e * kGdnC + ts], sv, su);
@@ -265,13 +269,20 @@ k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float
     }
     Us[ts * kGdnRB + r] = Ut[ts * kGdnRB + r] - su;
     __syncthreads();
-    const int jend = (ts & ~31) + 32;  // P is zero above its diagonal
-    for (int jj = 0; jj < jend; ++jj) sq = fmaf(Pt[jj * kGdnC + ts], Us[jj * kGdnRB + r], sq);
+    // P is zero above its diagonal: lanes of the first warp of a row stop at 32
+    if (ts < 32) {
+#pragma unroll 16
+      for (int jj = 0; jj < 32; ++jj) sq = fmaf(Pt[jj * kGdnC + ts], Us[jj * kGdnRB + r], sq);
+    } else {
+#pragma unroll 16
+      for (int jj = 0; jj < kGdnC; ++jj) sq = fmaf(Pt[jj * kGdnC + ts], Us[jj * kGdnRB + r], sq);
+    }
     Os[ts * kGdnRB + r] = sq;
     // S[r] = exp(g_last) S[r] + sum_t U[t][r] K~[t]
     for (int i = tid; i < kGdnRB * dk; i += kGdnThreads) {
       const int rr = i / dk, e = i - rr * dk;
       float acc = gl * Ss[i];
+#pragma unroll 16
       for (int t = 0; t < kGdnC; ++t) acc = fmaf(Us[t * kGdnRB + rr], Kt[t * dk + e], acc);
       Ss[i] = acc;
     }
@@ -284,6 +295,43 @@ k_gdn_scan(GdnPlan p, const float* __restrict__ ws, float* __restrict__ S, float
     }
   }
   for (int i = tid; i < kGdnRB * dk; i += kGdnThreads) Sg[i] = Ss[i];
+}
+
+template <int DK>
+static cudaError_t launch_gdn_dk(const GdnPlan& p, const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, float* S, float* o,
+                                 float* ws, size_t sp, size_t ss, int stages, dim3 gp, dim3 gs,
+                                 cudaStream_t s) {
+  cudaError_t e;
+  if (p.dtype == SDM_DTYPE_BF16) {
+    if ((e = cudaFuncSetAttribute(k_gdn_prep<__nv_bfloat16, DK>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, int(sp))) !=
+        cudaSuccess)
+      return e;
+    k_gdn_prep<__nv_bfloat16, DK><<<gp, kGdnThreads, sp, s>>>(
+        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, alpha,
+        beta, ws);
+  } else {
+    if ((e = cudaFuncSetAttribute(k_gdn_prep<float, DK>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, int(sp))) !=
+        cudaSuccess)
+      return e;
+    k_gdn_prep<float, DK><<<gp, kGdnThreads, sp, s>>>(p, (const float*)q, (const float*)k,
+                                                      (const float*)v, alpha, beta, ws);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (stages == 2) {
+    if ((e = cudaFuncSetAttribute(k_gdn_scan<DK, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(ss))) != cudaSuccess)
+      return e;
+    k_gdn_scan<DK, 2><<<gs, kGdnThreads, ss, s>>>(p, ws, S, o);
+  } else {
+    if ((e = cudaFuncSetAttribute(k_gdn_scan<DK, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(ss))) != cudaSuccess)
+      return e;
+    k_gdn_scan<DK, 1><<<gs, kGdnThreads, ss, s>>>(p, ws, S, o);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace sdm
@@ -321,32 +369,15 @@ extern "C" int sdm_gdn_forward(const void* q, const void* k, const void* v, cons
   const size_t ss = gdn_scan_smem(p.dk, stages);
   if (sp > 227 * 1024 || ss > 227 * 1024) return SDM_ERR_UNSUPPORTED;
   dim3 gp(p.nch, p.BH);
-  if (p.dtype == SDM_DTYPE_BF16) {
-    if (cudaFuncSetAttribute(k_gdn_prep<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(sp)) != cudaSuccess)
-      return SDM_ERR_CUDA;
-    k_gdn_prep<__nv_bfloat16><<<gp, kGdnThreads, sp, s>>>(
-        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, alpha,
-        beta, ws);
-  } else {
-    if (cudaFuncSetAttribute(k_gdn_prep<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(sp)) != cudaSuccess)
-      return SDM_ERR_CUDA;
-    k_gdn_prep<float><<<gp, kGdnThreads, sp, s>>>(p, (const float*)q, (const float*)k,
-                                                  (const float*)v, alpha, beta, ws);
-  }
-  if (cudaGetLastError() != cudaSuccess) return SDM_ERR_CUDA;
   dim3 gs(p.dv / kGdnRB, p.BH);
-  if (stages == 2) {
-    if (cudaFuncSetAttribute(k_gdn_scan<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(ss)) != cudaSuccess)
-      return SDM_ERR_CUDA;
-    k_gdn_scan<2><<<gs, kGdnThreads, ss, s>>>(p, ws, S_inout, o_out);
-  } else {
-    if (cudaFuncSetAttribute(k_gdn_scan<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(ss)) != cudaSuccess)
-      return SDM_ERR_CUDA;
-    k_gdn_scan<1><<<gs, kGdnThreads, ss, s>>>(p, ws, S_inout, o_out);
+  cudaError_t e;
+  switch (p.dk) {
+    case 16: e = launch_gdn_dk<16>(p, q, k, v, alpha, beta, S_inout, o_out, ws, sp, ss, stages, gp, gs, s); break;
+    case 32: e = launch_gdn_dk<32>(p, q, k, v, alpha, beta, S_inout, o_out, ws, sp, ss, stages, gp, gs, s); break;
+    case 64: e = launch_gdn_dk<64>(p, q, k, v, alpha, beta, S_inout, o_out, ws, sp, ss, stages, gp, gs, s); break;
+    case 128: e = launch_gdn_dk<128>(p, q, k, v, alpha, beta, S_inout, o_out, ws, sp, ss, stages, gp, gs, s); break;
+    default: return SDM_ERR_UNSUPPORTED;
   }
+  if (e != cudaSuccess) return SDM_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SDM_OK : SDM_ERR_CUDA;
 }
