@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--gdn", action="store_true",
                     help="time the dense Gated DeltaNet baseline at the matched size (d_k = W, "
                          "same B, H, T, d_v, gates) beside the SDM forward pass, and exit")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (sdm_backward) beside the forward pass on the "
+                         "workload, and exit")
     ap.add_argument("--probe-rows", action="store_true",
                     help="measure the HBM ceiling of random 256-byte row gathers and "
                          "read-modify-writes (the recurrence's access pattern) and exit")
@@ -699,6 +702,64 @@ def gdn_compare(cfg, steps, warmup):
             "steps": steps, "l2": "flushed before each step", "clocks": clk}
 
 
+def backward_bench(cfg, steps, warmup):
+    """sdm_backward on the workload (selections from sdm_select, random dL/do and
+    dL/dM_T), timed with CUDA events beside sdm_forward in the same process
+    (L2 flushed before each step)."""
+    import ctypes
+    import torch
+    import sparse_memory_linear_scoring_b200 as sdm
+    from synth import gen_inputs
+    dt = torch.bfloat16 if cfg.in_dtype == "bf16" else torch.float32
+    d = gen_inputs(cfg, device="cuda")
+    d = {n: (v.to(dt) if n in ("q", "k", "v", "C1", "C2") else v).contiguous()
+         for n, v in d.items()}
+    M0 = d["M0"]
+    lists = sdm.select(d["q"], d["k"], d["C1"], d["C2"], topk=cfg.k, W=cfg.W, R=cfg.R,
+                       d_v=cfg.d_v)
+    g = torch.Generator(device="cuda").manual_seed(0)
+    d_o = torch.randn(cfg.B, cfg.H, cfg.T, cfg.d_v, device="cuda", generator=g)
+    dM = torch.randn(M0.shape, device="cuda", generator=g)
+    dims = sdm.make_dims(**cfg.dims())
+    ws = torch.empty(int(sdm.load_library().sdm_backward_workspace_bytes(ctypes.byref(dims))),
+                     dtype=torch.uint8, device="cuda")
+    M = M0.clone()
+    o = torch.empty_like(d_o)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def time_it(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / steps
+
+    clocks = ClockSampler(_device_uuid(torch, torch.device("cuda")))
+    clocks.start()
+    bwd_ms = time_it(lambda: sdm.backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                                          d["C1"], d["C2"], M0, *lists, d_o, dM, topk=cfg.k,
+                                          workspace=ws))
+    fwd_ms = time_it(lambda: sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"],
+                                         d["C2"], M, topk=cfg.k, W=cfg.W, R=cfg.R, o=o))
+    clk = clocks.stop()
+    th = cfg.BH * cfg.T
+    return {"backward": "sdm_backward at the forward's selections (gradients of q, k, v, "
+                        "alpha, beta, C1, C2, M0)",
+            "workload": workload_desc(cfg), "backward_ms": bwd_ms,
+            "backward_token_heads_per_s": th / (bwd_ms / 1e3), "forward_ms": fwd_ms,
+            "backward_over_forward_time": bwd_ms / fwd_ms, "workspace_bytes": ws.numel(),
+            "steps": steps, "l2": "flushed before each step", "clocks": clk,
+            "device_status": sdm.device_status(ws)[0]}
+
+
 def main():
     args = parse()
     if args.decode:
@@ -707,6 +768,14 @@ def main():
         return 0
     if args.probe_rows:
         print(json.dumps(probe_rows()), flush=True)
+        return 0
+    if args.backward:
+        from synth import config as _config
+        cfg = _config(args.config)
+        if args.T > 0:
+            cfg = cfg.with_(T=args.T)
+        print(json.dumps(backward_bench(cfg, max(3, min(args.steps, 50)), max(2, args.warmup))),
+              flush=True)
         return 0
     if args.gdn:
         from synth import config as _config

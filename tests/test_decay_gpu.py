@@ -10,7 +10,8 @@ import torch
 
 import oracle
 import sparse_memory_linear_scoring_b200 as sdm
-from gpu_util import READ_BITS, REL_TOL, WRITE_BITS, head_rel_err, ncpu, np_inputs, to_device
+from gpu_util import (READ_BITS, REL_TOL, WRITE_BITS, elem_rel_err, head_rel_err, ncpu, np_inputs,
+                      report, to_device)
 from synth import config, gen_decay_rate, gen_inputs
 
 pytestmark = pytest.mark.gpu
@@ -42,8 +43,11 @@ def test_decay_rule_against_oracle(cfg):
         same &= eq
     clean = same.all(-1)
     assert clean.any()
-    eo = head_rel_err(o.cpu().numpy(), ref["o"], "decay o %s" % cfg.name)
-    eM = head_rel_err(M.cpu().numpy(), ref["M"], "decay M %s" % cfg.name)
+    og, Mg = o.cpu().numpy(), M.cpu().numpy()
+    eo = head_rel_err(og, ref["o"])
+    eM = head_rel_err(Mg, ref["M"])
+    report("decay o %s" % cfg.name, eo[clean], elem_rel_err(og, ref["o"])[clean])
+    report("decay M %s" % cfg.name, eM[clean], elem_rel_err(Mg, ref["M"])[clean])
     assert (eo[clean] <= REL_TOL).all(), eo
     assert (eM[clean] <= REL_TOL).all(), eM
     Mg, M0 = M.cpu().numpy(), inp["M0"].numpy()
