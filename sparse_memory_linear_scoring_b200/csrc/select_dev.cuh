@@ -1,5 +1,6 @@
 // select_dev.cuh -- warp-level exact top-k of (score, row) pairs held in
-// registers, used by the survivor top-k kernel and the single-step kernel.
+// registers, used by the tensor-core scoring epilogue and the survivor top-k
+// kernel.
 //
 // SDM summaries (gist.science 2607.07386), "Mecanismo Central" item 2: each
 // half keeps its top-k codebook rows, ordered by (score desc, row asc).  The
@@ -86,6 +87,94 @@ __device__ __forceinline__ void warp_gather_topk(const uint32_t (&key)[PL],
     if (take) out[base + __popc(mk & lt)] = (uint64_t(key[i]) << 32) | uint64_t(~row[i]);
     base += __popc(mk);
   }
+}
+
+// Scratch of warp_bucket_topk per warp: kSelBuckets cursors, kSelBuckets
+// bucket starts, then the staged 64-bit keys.
+constexpr int kSelBuckets = 64;
+constexpr int kSelHeadBytes = 2 * kSelBuckets * 4;
+
+// The k best of the c valid (key, row) entries held PL per lane (entry i*32 + l
+// in lane l; 1 <= k <= c; rows distinct), written to out[0..k) in (key desc,
+// row asc) order as (value bits, row) pairs, value = ord2f(key).
+//   1. The keys are counted into 64 buckets of the key range, bucket 0 holding
+//      the largest (bucket = (max - key) >> shift, monotone in the key).
+//   2. A warp scan of the counts gives every bucket's start in the output
+//      order and the bucket kb that holds the k-th largest.
+//   3. The entries of buckets 0..kb are staged, grouped by bucket.
+//   4. An entry's rank is its bucket's start plus the number of staged entries
+//      of its bucket that precede it; ranks below k are final positions.
+// A bucket holds a few entries unless the keys crowd together, so the rank
+// loops are short.  Returns false, writing nothing, if more than `cap` entries
+// would be staged (the caller then takes another path).
+template <int PL>
+__device__ __forceinline__ bool warp_bucket_topk(const uint32_t (&key)[PL],
+                                                 const uint32_t (&row)[PL], int c, int k,
+                                                 int* scr, uint64_t* stage, int cap, uint2* out) {
+  const int lane = threadIdx.x & 31;
+  int* cur = scr;                 // [64] counts, then cursors
+  int* start = scr + kSelBuckets; // [64] bucket starts
+  uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    if (i * 32 + lane < c) {
+      lo = min(lo, key[i]);
+      hi = max(hi, key[i]);
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  const uint32_t span = hi - lo;
+  const int nbits = 32 - __clz(span);  // span < 2^nbits
+  const int sh = nbits > 6 ? nbits - 6 : 0;
+  cur[lane] = 0;
+  cur[lane + 32] = 0;
+  __syncwarp();
+  int b[PL];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    b[i] = i * 32 + lane < c ? int((hi - key[i]) >> sh) : kSelBuckets;
+    if (b[i] < kSelBuckets) atomicAdd(&cur[b[i]], 1);
+  }
+  __syncwarp();
+  const int c0 = cur[2 * lane], c1 = cur[2 * lane + 1];
+  int incl = c0 + c1;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += y;
+  }
+  const int s0 = incl - c0 - c1, s1 = s0 + c0;  // starts of buckets 2 lane, 2 lane + 1
+  const unsigned ge = __ballot_sync(0xffffffffu, incl >= k);  // lane 31 holds c >= k
+  const int lk = __ffs(ge) - 1;
+  const int kb = 2 * lk + __shfl_sync(0xffffffffu, s1 >= k ? 0 : 1, lk);
+  const int nst = __shfl_sync(0xffffffffu, (kb & 1) ? incl : s1, kb >> 1);  // end of bucket kb
+  if (nst > cap) return false;
+  __syncwarp();
+  cur[2 * lane] = s0;
+  cur[2 * lane + 1] = s1;
+  start[2 * lane] = s0;
+  start[2 * lane + 1] = s1;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    if (b[i] <= kb) {
+      const int pos = atomicAdd(&cur[b[i]], 1);
+      stage[pos] = (uint64_t(key[i]) << 32) | uint64_t(~row[i]);
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    if (b[i] <= kb) {
+      const uint64_t me = (uint64_t(key[i]) << 32) | uint64_t(~row[i]);
+      const int bs = start[b[i]], be = cur[b[i]];
+      int rank = bs;
+      for (int j = bs; j < be; ++j) rank += stage[j] > me ? 1 : 0;
+      if (rank < k) out[rank] = make_uint2(__float_as_uint(ord2f(key[i])), row[i]);
+    }
+  }
+  return true;
 }
 
 }  // namespace sdm

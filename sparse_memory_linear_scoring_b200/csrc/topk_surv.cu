@@ -5,11 +5,13 @@
 // scoring kernel, a half-row's survivor list holds, unsorted, every score at
 // or above the row's threshold (between k and C entries); rows the filter could
 // not settle were re-scored exactly by the CUDA-core kernel (k entries, already
-// sorted).  One warp per half-row loads its list into registers, finds the
-// k-th largest score by a bitwise search over the order-preserving images,
-// gathers the k best (ties: lower row first), sorts them by (score desc, row
-// asc) and writes them back in place, so that the merge reads the first k
-// entries of every list, sorted, as it does after the other scoring kernels.
+// sorted).  One warp per half-row loads its list into registers and takes the
+// exact top-k of it by buckets of the key range (warp_bucket_topk), or, when
+// the buckets down to the k-th hold more entries than the staging area, by a
+// bitwise search for the k-th largest, a gather of the k best and a warp sort.
+// The k best are written back in place, sorted by (score desc, row asc), so
+// that the merge reads the first k entries of every list, sorted, as it does
+// after the other scoring kernels.
 #include "select_dev.cuh"
 
 namespace sdm {
@@ -22,7 +24,10 @@ k_topk_surv(Plan p, int tlen, int* __restrict__ cnt, uint2* __restrict__ surv, D
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K2 = next_pow2(p.k < 2 ? 2 : p.k);
-  uint64_t* sel = reinterpret_cast<uint64_t*>(smem) + size_t(warp) * K2;
+  const int cap = p.C > K2 ? p.C : K2;
+  unsigned char* wscr = smem + size_t(warp) * (kSelHeadBytes + 8 * size_t(cap));
+  int* scr = reinterpret_cast<int*>(wscr);
+  uint64_t* sel = reinterpret_cast<uint64_t*>(wscr + kSelHeadBytes);
   const int nrows = p.BH * tlen * 4;
   for (int w = blockIdx.x * kTopkWarps + warp; w < nrows; w += gridDim.x * kTopkWarps) {
     // w -> half-row (bh, tl, side, half) of the chunk
@@ -43,15 +48,18 @@ k_topk_surv(Plan p, int tlen, int* __restrict__ cnt, uint2* __restrict__ surv, D
       key[i] = f2ord(__uint_as_float(e.x));
       row[i] = e.y;
     }
-    const uint32_t thr = warp_kth_key<PL>(key, c, p.k);
-    warp_gather_topk<PL>(key, row, c, p.k, thr, sel);
-    __syncwarp();
-    for (int i = p.k + lane; i < K2; i += 32) sel[i] = 0;
-    __syncwarp();
-    warp_sort_desc(sel, K2);
-    for (int i = lane; i < p.k; i += 32) {
-      const uint64_t kv = sel[i];
-      list[i] = make_uint2(__float_as_uint(key_val(kv)), key_idx(kv));
+    __syncwarp();  // every lane has read the list before it is overwritten
+    if (!warp_bucket_topk<PL>(key, row, c, p.k, scr, sel, cap, list)) {
+      const uint32_t thr = warp_kth_key<PL>(key, c, p.k);
+      warp_gather_topk<PL>(key, row, c, p.k, thr, sel);
+      __syncwarp();
+      for (int i = p.k + lane; i < K2; i += 32) sel[i] = 0;
+      __syncwarp();
+      warp_sort_desc(sel, K2);
+      for (int i = lane; i < p.k; i += 32) {
+        const uint64_t kv = sel[i];
+        list[i] = make_uint2(__float_as_uint(key_val(kv)), key_idx(kv));
+      }
     }
     if (lane == 0) cnt[hr] = p.k;
     __syncwarp();
@@ -59,7 +67,9 @@ k_topk_surv(Plan p, int tlen, int* __restrict__ cnt, uint2* __restrict__ surv, D
 }
 
 size_t topk_surv_smem(const Plan& p) {
-  return size_t(kTopkWarps) * size_t(next_pow2(p.k < 2 ? 2 : p.k)) * 8;
+  const int K2 = next_pow2(p.k < 2 ? 2 : p.k);
+  const int cap = p.C > K2 ? p.C : K2;
+  return size_t(kTopkWarps) * (kSelHeadBytes + 8 * size_t(cap));
 }
 
 template <int PL>
