@@ -18,8 +18,9 @@
 //               row's scores and keep those above a threshold tau taken from
 //               the row's own score mean and deviation (first 512 columns);
 //               then, one warp per row, the exact top-k of the kept scores
-//               (bitwise search of the k-th, gather, warp sort), written
-//               sorted by (score desc, row asc).
+//               (64 buckets of the key range, a warp scan of their counts,
+//               ranks within the buckets down to the k-th), written sorted by
+//               (score desc, row asc).
 // A row whose kept count falls outside [k, capacity] (or whose scores do not
 // spread) is queued for the exact CUDA-core path instead, so the result is
 // exact for any input.  Every mbarrier wait is bounded: on a timeout the CTA
@@ -44,6 +45,10 @@ constexpr int kQ = 4;                // epilogue threads per token row
 constexpr int kEpiThreads = kQ * kTileM;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+#ifndef SDM_POLL_SLEEP_NS
+#define SDM_POLL_SLEEP_NS 32
+#endif
+constexpr unsigned kPollSleepNs = SDM_POLL_SLEEP_NS;  // pause between mbarrier polls
 constexpr uint32_t kATileBytes = kTileM * 128;   // one 64-column chunk of the token tile
 constexpr uint32_t kBTileBytes = kTileN * 128;   // one 64-column chunk of a codebook tile
 
@@ -60,15 +65,27 @@ struct TcArgs {
 // Per-row survivor lists are row-major with one element of padding (row
 // stride C + 1 floats, C + 2 row numbers), so that the filter's appends (one
 // lane per row) and the selection's reads (one warp per row) both spread over
-// the banks.
+// the banks.  The selection's per-warp scratch (bucket counters, then staged
+// 64-bit keys) has its own area: the token tile and the codebook ring are
+// already being refilled for the CTA's next work item while it runs.
 struct TcLayout {
-  uint32_t a, b, vals, idx, rows, bars, total;
-  int nkc;
+  uint32_t a, b, vals, idx, rows, sel, bars, total;
+  int nkc, cap;
 };
+
+// Staged entries per warp: the k best plus 24 (the bucket holding the k-th),
+// and at least the fallback's sort buffer (next_pow2(k) keys); at most C.
+__host__ __device__ inline int sel_cap(int C, int k) {
+  const int k2 = next_pow2(k < 2 ? 2 : k);
+  int cap = k + 24 > k2 ? k + 24 : k2;
+  cap = (cap + 7) & ~7;
+  return cap < C ? cap : (C > k2 ? C : k2);
+}
 
 __host__ __device__ inline TcLayout tc_layout(const Plan& p) {
   TcLayout L;
   L.nkc = p.dh / kKAtom;
+  L.cap = sel_cap(p.C, p.k);
   uint32_t o = 0;
   L.a = o; o += L.nkc * kATileBytes;
   L.b = o; o += 2 * L.nkc * kBTileBytes;
@@ -76,16 +93,10 @@ __host__ __device__ inline TcLayout tc_layout(const Plan& p) {
   L.idx = o; o += uint32_t(p.C + 2) * kTileM * 2;
   o = (o + 15) & ~15u;
   L.rows = o; o += (2 + 2 * kQ) * kTileM * 4;  // per-row count, go flag, partial stats
-  o = (o + 15) & ~15u;
+  L.sel = o; o += uint32_t(kEpiThreads / 32) * uint32_t(kSelHeadBytes + 8 * L.cap);
   L.bars = o; o += 16 * 8;  // mbarriers, TMEM address, abort flags
   L.total = o + 1024;  // slack for 1024-byte alignment of the dynamic base
   return L;
-}
-
-// The selection's per-warp sort buffers reuse the token tile and codebook
-// ring once every MMA has completed: 16 warps x next_pow2(k) 64-bit keys.
-__host__ __device__ inline bool sort_area_fits(const TcLayout& L, int k) {
-  return uint32_t(kEpiThreads / 32) * uint32_t(next_pow2(k < 2 ? 2 : k)) * 8u <= L.vals - L.a;
 }
 
 // ---- PTX wrappers -------------------------------------------------------------
@@ -113,6 +124,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait; false when it timed out or another role already gave up.
+// Between polls the warp sleeps briefly, so that waiting warps leave the issue
+// slots to the epilogue warps that share their SM sub-partition.
 __device__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
   const long long t0 = clock64();
   while (!mbar_test(b, parity)) {
@@ -121,6 +134,7 @@ __device__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag
       *abort_flag = 1;
       return false;
     }
+    __nanosleep(kPollSleepNs);
   }
   return true;
 }
@@ -207,20 +221,23 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
   float* vals = reinterpret_cast<float*>(smem + L.vals);        // [128][C + 1]
   uint16_t* idxs = reinterpret_cast<uint16_t*>(smem + L.idx);   // [128][C + 2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* full = bars;       // [2] TMA -> MMA
+  uint64_t* full = bars;       // [2] TMA -> MMA (codebook ring)
   uint64_t* empty = bars + 2;  // [2] MMA -> TMA
-  uint64_t* a_full = bars + 4;
-  uint64_t* tfull = bars + 5;  // [2] MMA -> epilogue
-  uint64_t* tempty = bars + 7; // [2] epilogue -> MMA
-  uint64_t* drain = bars + 9;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 10);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  uint64_t* a_full = bars + 4; // token tile landed
+  uint64_t* a_empty = bars + 5;// token tile consumed by every MMA of its item
+  uint64_t* tfull = bars + 6;  // [2] MMA -> epilogue
+  uint64_t* tempty = bars + 8; // [2] epilogue -> MMA
+  uint64_t* drain = bars + 10;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
+  volatile int* epi_abort = reinterpret_cast<volatile int*>(bars + 13);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, bh = blockIdx.y, side = blockIdx.z >> 1, half = blockIdx.z & 1;
-  const int h = bh % p.H;
   const int ntiles = p.n / kTileN;
   const int nk = p.dh / 16;
+  // work items: (token tile, head, side, half), side/half fastest
+  const int ntt = (a.tlen + kTileM - 1) / kTileM;
+  const int nitems = ntt * p.BH * 4;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -230,9 +247,10 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
       mbar_init(&tempty[i], kEpiThreads);
     }
     mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *reinterpret_cast<volatile int*>(bars + 12) = 0;
+    *epi_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -248,56 +266,80 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer: each item's token tile, then its codebook
+    // tiles through the ring (gb counts the ring's fills over all items)
     if (lane == 0) {
-      const CUtensorMap* mx = side ? &mq : &mk;
-      const CUtensorMap* mc = half ? &mc2 : &mc1;
-      tma_prefetch(mx);
-      tma_prefetch(mc);
-      const int row0 = bh * p.T + a.t0 + tile * kTileM;
-      mbar_expect_tx(a_full, L.nkc * kATileBytes);
-      for (int kc = 0; kc < L.nkc; ++kc)
-        tma_load_2d(mx, a_full, sA + kc * kATileBytes, half * p.dh + kc * kKAtom, row0);
-      int issued = 0;
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag)) break;
-        mbar_expect_tx(&full[s], L.nkc * kBTileBytes);
+      tma_prefetch(&mq);
+      tma_prefetch(&mk);
+      tma_prefetch(&mc1);
+      tma_prefetch(&mc2);
+      int gb = 0, na = 0;
+      bool live = true;
+      for (int w = blockIdx.x, i = 0; w < nitems && live; w += gridDim.x, ++i) {
+        const int z = w & 3, rest = w >> 2;
+        const int tile = rest % ntt, bh = rest / ntt, side = z >> 1, half = z & 1;
+        const CUtensorMap* mx = side ? &mq : &mk;
+        const CUtensorMap* mc = half ? &mc2 : &mc1;
+        if (i >= 1 && !mbar_wait(a_empty, (i - 1) & 1, abort_flag)) break;
+        const int row0 = bh * p.T + a.t0 + tile * kTileM;
+        mbar_expect_tx(a_full, L.nkc * kATileBytes);
         for (int kc = 0; kc < L.nkc; ++kc)
-          tma_load_2d(mc, &full[s], sB + (s * L.nkc + kc) * kBTileBytes, kc * kKAtom,
-                      h * p.n + j * kTileN);
-        ++issued;
+          tma_load_2d(mx, a_full, sA + kc * kATileBytes, half * p.dh + kc * kKAtom, row0);
+        ++na;
+        const int h = bh % p.H;
+        for (int j = 0; j < ntiles; ++j, ++gb) {
+          const int s = gb & 1;
+          if (gb >= 2 && !mbar_wait(&empty[s], ((gb >> 1) & 1) ^ 1, abort_flag)) {
+            live = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], L.nkc * kBTileBytes);
+          for (int kc = 0; kc < L.nkc; ++kc)
+            tma_load_2d(mc, &full[s], sB + (s * L.nkc + kc) * kBTileBytes, kc * kKAtom,
+                        h * p.n + j * kTileN);
+        }
       }
       // on abort: let the copies already issued land before the CTA leaves
+      // (the last fill of each barrier: none of them has advanced past it)
       if (*abort_flag) {
         volatile int never = 0;
-        mbar_wait(a_full, 0, &never);
-        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-          mbar_wait(&full[j & 1], (j >> 1) & 1, &never);
+        if (na > 0) mbar_wait(a_full, (na - 1) & 1, &never);
+        for (int g = (gb > 2 ? gb - 2 : 0); g < gb; ++g)
+          mbar_wait(&full[g & 1], (g >> 1) & 1, &never);
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer (gb: ring fills consumed, gt: TMEM buffers filled)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(kTileM, kTileN);
-      int issued = 0;
-      if (mbar_wait(a_full, 0, abort_flag)) {
-        for (int j = 0; j < ntiles; ++j) {
-          const int s = j & 1;
-          if (!mbar_wait(&full[s], (j >> 1) & 1, abort_flag)) break;
-          if (j >= 2 && !mbar_wait(&tempty[s], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+      // this CTA's items and ring fills: the producer waits for the release of
+      // every fill but the last two, so only those releases are committed
+      const int my_items = blockIdx.x < nitems ? (nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      const int nfill = my_items * ntiles;
+      int gb = 0, gt = 0, issued = 0;
+      bool live = true;
+      for (int w = blockIdx.x, i = 0; w < nitems && live; w += gridDim.x, ++i) {
+        if (!mbar_wait(a_full, i & 1, abort_flag)) break;
+        for (int j = 0; j < ntiles; ++j, ++gb, ++gt) {
+          const int s = gb & 1, buf = gt & 1;
+          if (!mbar_wait(&full[s], (gb >> 1) & 1, abort_flag) ||
+              (gt >= 2 && !mbar_wait(&tempty[buf], ((gt >> 1) & 1) ^ 1, abort_flag))) {
+            live = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t d = tmem + uint32_t(s * kTileN);
+          const uint32_t d = tmem + uint32_t(buf * kTileN);
           for (int kk = 0; kk < nk; ++kk) {
-            const int kc = kk >> 2, w = kk & 3;
-            const uint64_t ad = sdesc(su32(sA + kc * kATileBytes + w * 32));
-            const uint64_t bd = sdesc(su32(sB + (s * L.nkc + kc) * kBTileBytes + w * 32));
+            const int kc = kk >> 2, ww = kk & 3;
+            const uint64_t ad = sdesc(su32(sA + kc * kATileBytes + ww * 32));
+            const uint64_t bd = sdesc(su32(sB + (s * L.nkc + kc) * kBTileBytes + ww * 32));
             umma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&empty[s]);
-          umma_commit(&tfull[s]);
+          if (gb + 2 < nfill) umma_commit(&empty[s]);
+          umma_commit(&tfull[buf]);
           ++issued;
         }
+        if (live && i + 1 < my_items) umma_commit(a_empty);
       }
       if (*abort_flag && issued > 0) {
         // wait (bounded) for the MMAs already issued before TMEM is freed
@@ -311,142 +353,153 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
     const int q4 = warp & 3;
     const int sub = (warp - 2) >> 2;  // which kCols-column slice of every tile
     const int row = q4 * 32 + lane;
-    const int tl = tile * kTileM + row;
-    const bool valid = tl < a.tlen;
     const uint32_t tbase = tmem + (uint32_t(q4 * 32) << 16);
     const int C = p.C;
+    const int k = p.k;
     constexpr int kCols = kTileN / kQ;
     int* rcnt = reinterpret_cast<int*>(smem + L.rows);      // [128] kept count
     int* rgo = rcnt + kTileM;                               // [128] row settled here
     float* rst = reinterpret_cast<float*>(rgo + kTileM);    // [2][kQ][128] sum, sq
-    volatile int* epi_abort = reinterpret_cast<volatile int*>(bars + 12);
-    float v[32];
-    if (sub == 0) rcnt[row] = 0;
-    // statistics of the first (up to) two tiles
-    const int nstat = ntiles < 2 ? ntiles : 2;
-    float sum = 0.f, sq = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nstat && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&tfull[j], 0, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < kCols / 32; ++c) {
-        tmem_ld32(tbase + uint32_t(j * kTileN + sub * kCols + c * 32), v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sum += v[i];
-          sq = fmaf(v[i], v[i], sq);
-        }
-      }
-    }
-    if (!ok) *epi_abort = 1;
-    rst[(0 * kQ + sub) * kTileM + row] = sum;
-    rst[(1 * kQ + sub) * kTileM + row] = sq;
-    epi_sync();
-    ok = !*epi_abort;
+    const int ew = warp - 2;
+    const int K2 = next_pow2(k < 2 ? 2 : k);
+    unsigned char* wscr = smem + L.sel + size_t(ew) * size_t(kSelHeadBytes + 8 * L.cap);
+    int* scr = reinterpret_cast<int*>(wscr);
+    uint64_t* stage = reinterpret_cast<uint64_t*>(wscr + kSelHeadBytes);
     const bool keep_all = !(a.z > -1e30f);
-    float tau = -INFINITY;
-    bool redo = false;
-    {
-      float S = 0.f, S2 = 0.f;
-#pragma unroll
-      for (int j = 0; j < kQ; ++j) {
-        S += rst[(0 * kQ + j) * kTileM + row];
-        S2 += rst[(1 * kQ + j) * kTileM + row];
-      }
-      const float m = float(nstat * kTileN);
-      const float mu = S / m;
-      const float sd = sqrtf(fmaxf(S2 / m - mu * mu, 0.f));
-      if (!keep_all) tau = mu + a.z * sd;
-      redo = !keep_all && !(sd > 0.f);
-      // rows past the end of the chunk keep nothing, so that a warp whose rows
-      // are all past it skips the appends (single steps, ragged last tiles)
-      if (!valid) tau = INFINITY;
-    }
-    // filter: append the kept scores of this thread's columns to the row's list
-    float* vrow = vals + row * (C + 1);
-    uint16_t* irow = idxs + row * (C + 2);
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int s = j & 1;
-      if (j >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[s], (j >> 1) & 1, abort_flag));
+    const int nstat = ntiles < 2 ? ntiles : 2;
+    bool ok = true;
+    float v[32];
+    for (int w = blockIdx.x, i = 0; w < nitems; w += gridDim.x, ++i) {
+      const int z = w & 3, rest = w >> 2;
+      const int tile = rest % ntt, bh = rest / ntt, side = z >> 1, half = z & 1;
+      const int tl = tile * kTileM + row;
+      const bool valid = tl < a.tlen;
+      const int gt0 = i * ntiles;  // TMEM buffer fills before this item's
+      if (sub == 0) rcnt[row] = 0;
+      // statistics of the first (up to) two tiles
+      float sum = 0.f, sq = 0.f;
+      for (int j = 0; j < nstat && ok; ++j) {
+        const int g = gt0 + j;
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[g & 1], (g >> 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
-      }
 #pragma unroll 1
-      for (int c = 0; c < kCols / 32; ++c) {
-        tmem_ld32(tbase + uint32_t(s * kTileN + sub * kCols + c * 32), v);
-        const int col0 = j * kTileN + sub * kCols + c * 32;
-        uint32_t mask = 0;
+        for (int c = 0; c < kCols / 32; ++c) {
+          tmem_ld32(tbase + uint32_t((g & 1) * kTileN + sub * kCols + c * 32), v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mask |= (v[i] >= tau ? 1u : 0u) << i;
-        if (mask) {
-          int pos = atomicAdd(&rcnt[row], __popc(mask));
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if ((mask >> i) & 1u) {
-              if (pos < C) {
-                vrow[pos] = v[i];
-                irow[pos] = uint16_t(col0 + i);
-              }
-              ++pos;
-            }
+          for (int ii = 0; ii < 32; ++ii) {
+            sum += v[ii];
+            sq = fmaf(v[ii], v[ii], sq);
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[s]);
-    }
-    if (!ok) *epi_abort = 1;
-    epi_sync();
-    ok = !*epi_abort;
-    if (!ok && threadIdx.x == 64) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
-    const int k = p.k;
-    if (sub == 0) {
-      const int cnt = rcnt[row];
-      const bool go = ok && valid && !redo && cnt >= k && cnt <= C;
-      rgo[row] = go ? 1 : 0;
-      // every valid row this CTA does not settle -- including all of them after
-      // a timed-out wait -- is re-scored exactly, so no later kernel reads a
-      // list this call never wrote
-      const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
-      if (valid && !go) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
-    }
-    epi_sync();
-    // exact top-k of each settled row's kept scores, one warp per row: the
-    // k-th largest order-preserving image by a bitwise search, the k best
-    // gathered (ties: lowest codebook row), sorted by (score desc, row asc)
-    // and written to the survivor list.  Every MMA has completed (each thread
-    // waited for the last tile), so the token tile and codebook ring hold the
-    // warps' sort buffers.
-    const int ew = warp - 2;
-    const int K2 = next_pow2(k < 2 ? 2 : k);
-    uint64_t* sbuf = reinterpret_cast<uint64_t*>(smem + L.a) + size_t(ew) * K2;
-    for (int r = ew; r < kTileM; r += kEpiThreads / 32) {
-      if (!rgo[r]) continue;
-      const int cnt = rcnt[r];
-      const float* vr = vals + r * (C + 1);
-      const uint16_t* ir = idxs + r * (C + 2);
-      uint32_t key[PL], rw[PL];
+      if (!ok) *epi_abort = 1;
+      rst[(0 * kQ + sub) * kTileM + row] = sum;
+      rst[(1 * kQ + sub) * kTileM + row] = sq;
+      epi_sync();
+      ok = !*epi_abort;
+      float tau = -INFINITY;
+      bool redo = false;
+      {
+        float S = 0.f, S2 = 0.f;
 #pragma unroll
-      for (int i = 0; i < PL; ++i) {
-        const int jj = i * 32 + lane;
-        key[i] = jj < cnt ? f2ord(vr[jj]) : 0u;
-        rw[i] = jj < cnt ? uint32_t(ir[jj]) : 0u;
+        for (int j = 0; j < kQ; ++j) {
+          S += rst[(0 * kQ + j) * kTileM + row];
+          S2 += rst[(1 * kQ + j) * kTileM + row];
+        }
+        const float m = float(nstat * kTileN);
+        const float mu = S / m;
+        const float sd = sqrtf(fmaxf(S2 / m - mu * mu, 0.f));
+        if (!keep_all) tau = mu + a.z * sd;
+        redo = !keep_all && !(sd > 0.f);
+        // rows past the end of the chunk keep nothing, so that a warp whose rows
+        // are all past it skips the appends (single steps, ragged last tiles)
+        if (!valid) tau = INFINITY;
       }
-      const uint32_t thr = warp_kth_key<PL>(key, cnt, k);
-      warp_gather_topk<PL>(key, rw, cnt, k, thr, sbuf);
-      __syncwarp();
-      for (int i = k + lane; i < K2; i += 32) sbuf[i] = 0;
-      __syncwarp();
-      warp_sort_desc(sbuf, K2);
-      const size_t hr = (size_t(bh) * p.Tc + tile * kTileM + r) * 4 + side * 2 + half;
-      uint2* g = a.surv + hr * C;
-      for (int i = lane; i < k; i += 32)
-        g[i] = make_uint2(__float_as_uint(key_val(sbuf[i])), key_idx(sbuf[i]));
-      if (lane == 0) a.cnt[hr] = k;
-      __syncwarp();
+      // filter: append the kept scores of this thread's columns to the row's list
+      float* vrow = vals + row * (C + 1);
+      uint16_t* irow = idxs + row * (C + 2);
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int g = gt0 + j, buf = g & 1;
+        if (j >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (g >> 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll 1
+        for (int c = 0; c < kCols / 32; ++c) {
+          tmem_ld32(tbase + uint32_t(buf * kTileN + sub * kCols + c * 32), v);
+          const int col0 = j * kTileN + sub * kCols + c * 32;
+          uint32_t mask = 0;
+#pragma unroll
+          for (int ii = 0; ii < 32; ++ii) mask |= (v[ii] >= tau ? 1u : 0u) << ii;
+          if (mask) {
+            int pos = atomicAdd(&rcnt[row], __popc(mask));
+#pragma unroll
+            for (int ii = 0; ii < 32; ++ii) {
+              if ((mask >> ii) & 1u) {
+                if (pos < C) {
+                  vrow[pos] = v[ii];
+                  irow[pos] = uint16_t(col0 + ii);
+                }
+                ++pos;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+      }
+      if (!ok) *epi_abort = 1;
+      epi_sync();
+      ok = !*epi_abort;
+      if (!ok && threadIdx.x == 64) dev_flag(a.st, SDM_DEV_TIMEOUT, blockIdx.x);
+      if (sub == 0) {
+        const int cnt = rcnt[row];
+        const bool go = ok && valid && !redo && cnt >= k && cnt <= C;
+        rgo[row] = go ? 1 : 0;
+        // every valid row this CTA does not settle -- including all of them
+        // after a timed-out wait -- is re-scored exactly, so no later kernel
+        // reads a list this call never wrote
+        const size_t hr = (size_t(bh) * p.Tc + tl) * 4 + side * 2 + half;
+        if (valid && !go) a.redo[atomicAdd(&a.st->redo, 1)] = int(hr);
+      }
+      epi_sync();
+      // exact top-k of each settled row's kept scores, one warp per row, sorted
+      // by (score desc, row asc) and written to the survivor list: by buckets
+      // of the key range (warp_bucket_topk), or -- when the buckets down to the
+      // k-th hold more entries than the staging area -- by a bitwise search for
+      // the k-th largest, a gather of the k best and a warp sort.  Meanwhile the
+      // producer and the MMA issuer already work on the CTA's next item.
+      for (int r = ew; r < kTileM; r += kEpiThreads / 32) {
+        if (!rgo[r]) continue;
+        const int cnt = rcnt[r];
+        const float* vr = vals + r * (C + 1);
+        const uint16_t* ir = idxs + r * (C + 2);
+        uint32_t key[PL], rw[PL];
+#pragma unroll
+        for (int ii = 0; ii < PL; ++ii) {
+          const int jj = ii * 32 + lane;
+          key[ii] = jj < cnt ? f2ord(vr[jj]) : 0u;
+          rw[ii] = jj < cnt ? uint32_t(ir[jj]) : 0u;
+        }
+        const size_t hr = (size_t(bh) * p.Tc + tile * kTileM + r) * 4 + side * 2 + half;
+        uint2* g = a.surv + hr * C;
+        if (!warp_bucket_topk<PL>(key, rw, cnt, k, scr, stage, L.cap, g)) {
+          const uint32_t thr = warp_kth_key<PL>(key, cnt, k);
+          warp_gather_topk<PL>(key, rw, cnt, k, thr, stage);
+          __syncwarp();
+          for (int ii = k + lane; ii < K2; ii += 32) stage[ii] = 0;
+          __syncwarp();
+          warp_sort_desc(stage, K2);
+          for (int ii = lane; ii < k; ii += 32)
+            g[ii] = make_uint2(__float_as_uint(key_val(stage[ii])), key_idx(stage[ii]));
+        }
+        if (lane == 0) a.cnt[hr] = k;
+        __syncwarp();
+      }
+      // the next item's counts, statistics and lists overwrite this one's
+      epi_sync();
     }
   }
   tc_fence_before();
@@ -783,11 +836,11 @@ int score_tc_mode(const sdm_dims* d) {
   Plan tmp;
   tmp.dh = dh;
   tmp.C = score_tc_capacity(d, 1);
+  tmp.k = d->k;
   tmp.tc = 1;
   const TcLayout L = tc_layout(tmp);
-  // per-row bucket counts and offsets are packed bytes: the capacity stays below 256
-  const bool m1 = d->n_sub % kTileN == 0 && tmp.C <= 8 * 32 && L.total <= 227 * 1024 &&
-                  sort_area_fits(L, d->k);
+  // the selection holds a row's kept scores in registers, at most 8 per lane
+  const bool m1 = d->n_sub % kTileN == 0 && tmp.C <= 8 * 32 && L.total <= 227 * 1024;
   tmp.tc = 2;
   tmp.C = score_tc_capacity(d, 2);
   const bool m2 = tc_layout_f(tmp).total <= 227 * 1024;
@@ -826,21 +879,29 @@ cudaError_t launch_score_tc(const Plan& p, const void* q, const void* k, const v
     if (e != cudaSuccess) return e;
     k_score_tc_filter<<<grid, kThreadsF, smem, s>>>(mq, mk, mc1, mc2, a);
   } else {
+    // persistent: one CTA per SM (its shared memory), each walking the work
+    // items (token tile, head, side, half) with a stride of the grid
+    int dev = 0, nsm = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long nitems = (long long)grid.x * p.BH * 4;
+    const int pgrid = int(nitems < nsm ? nitems : nsm);
     if (p.C <= 4 * 32) {
       e = cudaFuncSetAttribute(k_score_tc<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(smem));
       if (e != cudaSuccess) return e;
-      k_score_tc<4><<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+      k_score_tc<4><<<pgrid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
     } else if (p.C <= 5 * 32) {
       e = cudaFuncSetAttribute(k_score_tc<5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(smem));
       if (e != cudaSuccess) return e;
-      k_score_tc<5><<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+      k_score_tc<5><<<pgrid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
     } else {
       e = cudaFuncSetAttribute(k_score_tc<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(smem));
       if (e != cudaSuccess) return e;
-      k_score_tc<8><<<grid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
+      k_score_tc<8><<<pgrid, kThreads, smem, s>>>(mq, mk, mc1, mc2, a);
     }
   }
   return cudaGetLastError();
