@@ -47,8 +47,9 @@ __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   size_t o = 0;
   L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR + 2 * p.k) * 4);
   L.uni = o;
-  // h1, h2 [Sk], sel [Ss] (64-bit); cand, cell [Sc], select scratch [2 Sc] (32-bit)
-  L.per_warp = size_t(2 * L.Sk + L.Ss) * 8 + size_t(4 * L.Sc) * 4;
+  // h1, h2 [Sk], sel [Ss] (64-bit); cand, cell [Sc], select scratch [2 Sc],
+  // bucket counts [64] (32-bit)
+  L.per_warp = size_t(2 * L.Sk + L.Ss) * 8 + size_t(4 * L.Sc + 64) * 4;
   o += L.per_warp * warps;
   L.total = al16(o);
   return L;
@@ -211,7 +212,7 @@ __device__ inline uint32_t warp_select32(const uint32_t* cand, int n, int r, uin
 __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
                           int n_sel, const uint32_t* stair, int n_stair, const uint32_t* front,
                           int nf, const int* ediv, uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* cell,
-                          uint32_t* alt, uint64_t* sel, bool sorted, float* w_out,
+                          uint32_t* alt, int* hist, uint64_t* sel, bool sorted, float* w_out,
                           uint32_t* slot_out, DevStatus* st, int info, bool sigmoid_w = false) {
   const int lane = threadIdx.x & 31;
   if (c1 < p.k || c1 > p.C || c2 < p.k || c2 > p.C) {
@@ -238,7 +239,14 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   lb = __reduce_max_sync(0xffffffffu, lb);
   // candidates: the staircase cells scoring >= lb (ordered 32-bit images of the
   // float32 sums) and their cells; they include every staircase cell that
-  // scores >= the n_sel-th best
+  // scores >= the n_sel-th best, so nc >= n_sel.  Each is also counted into one
+  // of 64 buckets of [lb, hi] (hi: cell (0, 0), the best), bucket 0 the highest.
+  const uint32_t hi = f2ord(hval(h1[0]) + hval(h2[0]));
+  const int nbits = 32 - __clz(hi - lb);  // hi - lb < 2^nbits
+  const int sh = nbits > 6 ? nbits - 6 : 0;
+  hist[lane] = 0;
+  hist[lane + 32] = 0;
+  __syncwarp();
   int nc = 0;
   for (int i0 = 0; i0 < n_stair; i0 += 32) {
     const int i = i0 + lane;
@@ -253,11 +261,48 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
       const int pos = nc + __popc(m & lanemask_lt());
       cand[pos] = x;
       cell[pos] = ab;
+      atomicAdd(&hist[(hi - x) >> sh], 1);
     }
     nc += __popc(m);
   }
   __syncwarp();
-  const uint32_t vstar = warp_select32(cand, nc, n_sel, alt, alt + (nc + 31) / 32 * 32);
+  // the n_sel-th best: a warp scan of the bucket counts finds the bucket kb
+  // that holds it and its rank r there; a bucket of at most 32 entries is
+  // sorted across the warp, a larger one (crowded scores) goes to quickselect
+  uint32_t vstar;
+  {
+    const int c0 = hist[2 * lane], c1 = hist[2 * lane + 1];
+    int incl = c0 + c1;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += y;
+    }
+    const int s0 = incl - c0 - c1, s1 = s0 + c0;
+    const int lk = __ffs(__ballot_sync(0xffffffffu, incl >= n_sel)) - 1;
+    const int odd = __shfl_sync(0xffffffffu, s1 >= n_sel ? 0 : 1, lk);
+    const uint32_t kb = uint32_t(2 * lk + odd);
+    const int kb0 = __shfl_sync(0xffffffffu, odd ? s1 : s0, lk);
+    const int kb1 = __shfl_sync(0xffffffffu, odd ? incl : s1, lk);
+    if (kb1 - kb0 <= 32) {
+      int nb = 0;
+      for (int i0 = 0; i0 < nc; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t x = i < nc ? cand[i] : 0u;
+        const bool in = i < nc && ((hi - x) >> sh) == kb;
+        const unsigned m = __ballot_sync(0xffffffffu, in);
+        if (in) alt[nb + __popc(m & lanemask_lt())] = x;
+        nb += __popc(m);
+      }
+      __syncwarp();
+      uint32_t y = lane < kb1 - kb0 ? alt[lane] : 0u;
+      y = warp_sort32_desc_u32(y);
+      vstar = __shfl_sync(0xffffffffu, y, n_sel - kb0 - 1);
+      __syncwarp();
+    } else {
+      vstar = warp_select32(cand, nc, n_sel, alt, alt + (nc + 31) / 32 * 32);
+    }
+  }
   // exact when every candidate outside the staircase scores strictly below the
   // n_sel-th and no other candidate ties it
   int n_gt = 0, n_eq = 0;

@@ -9,7 +9,8 @@
 //
 // Merge (one warp per (step, side)): the half lists arrive sorted; evaluate the
 // "staircase" candidates (a, b) with (a+1)(b+1) <= n_sel (a, b = ranks in the
-// two halves) and select the n_sel best by quickselect.  This is exact when every
+// two halves) and select the n_sel best (64 buckets of the score range, then a
+// warp sort of the bucket that holds the n_sel-th, or quickselect).  This is exact when every
 // candidate outside the staircase scores strictly below the n_sel-th: the
 // largest outside score is attained on the staircase's frontier (row a, column
 // bmax(a)), since sums fall along each row; if the frontier check fails, an
@@ -83,6 +84,7 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   uint32_t* cand = reinterpret_cast<uint32_t*>(sel + L.Ss);
   uint32_t* cell = cand + L.Sc;
   uint32_t* alt = cell + L.Sc;
+  int* hist = reinterpret_cast<int*>(alt + 2 * L.Sc);
   for (int pi = warp; pi < 2 * np; pi += kMergeWarps) {
     const int tc = s0 + (pi >> 1), side = pi & 1;
     const size_t hr = (size_t(bh) * p.Tc + tc) * 4 + side * 2;
@@ -93,7 +95,7 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
     merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
               io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
               side ? frontR : frontW, side ? p.nfR : p.nfW, side ? edivR : edivW, h1, h2, cand,
-              cell, alt, sel,
+              cell, alt, hist, sel,
               io.sorted != 0, w_out, s_out, st, int(hr), p.rule == 1 && side == 0);
   }
 }

@@ -330,11 +330,12 @@ __global__ void __launch_bounds__(kStepThreads, 1) k_step(Plan p, StepIO io) {
       uint32_t* cand = reinterpret_cast<uint32_t*>(sel + L.ML.Ss);
       uint32_t* cell = cand + L.ML.Sc;
       uint32_t* alt = cell + L.ML.Sc;
+      int* hist = reinterpret_cast<int*>(alt + 2 * L.ML.Sc);
       float* w_out = selw + (side ? p.W : 0);
       uint32_t* s_out = sels + (side ? p.W : 0);
       merge_one(p, hl + size_t(side * 2) * K2, k, hl + size_t(side * 2 + 1) * K2, k, n_sel,
                 side ? stairR : stairW, side ? p.ncR : p.ncW, side ? frontR : frontW,
-                side ? p.nfR : p.nfW, side ? edivR : edivW, h1, h2, cand, cell, alt, sel, lists,
+                side ? p.nfR : p.nfW, side ? edivR : edivW, h1, h2, cand, cell, alt, hist, sel, lists,
                 w_out, s_out, st, t);
       if (lists) {
         int32_t* gi = (side ? io.idx_r : io.idx_w) + row * n_sel;
