@@ -199,6 +199,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Predicated stores (no branch): write x at the address when `on` is nonzero.
+__device__ __forceinline__ void sts_f32_if(uint32_t a, float x, uint32_t on) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p st.shared.f32 [%0], %1;\n}\n"
+               ::"r"(a), "f"(x), "r"(on));
+}
+__device__ __forceinline__ void sts_u16_if(uint32_t a, uint16_t x, uint32_t on) {
+  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p st.shared.u16 [%0], %1;\n}\n"
+               ::"r"(a), "h"(x), "r"(on));
+}
+
 // named barrier of the epilogue warps
 __device__ __forceinline__ void epi_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
@@ -433,8 +443,22 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
           uint32_t mask = 0;
 #pragma unroll
           for (int ii = 0; ii < 32; ++ii) mask |= (v[ii] >= tau ? 1u : 0u) << ii;
-          if (mask) {
-            int pos = atomicAdd(&rcnt[row], __popc(mask));
+          // reserve the places (one shared atomic), then append with predicated
+          // stores: no branch per score, so the warp does not diverge
+          const int nk = __popc(mask);
+          const int pos0 = atomicAdd(&rcnt[row], nk);
+          if (pos0 + nk <= C) {
+            uint32_t av = su32(vrow + pos0), ai = su32(irow + pos0);
+#pragma unroll
+            for (int ii = 0; ii < 32; ++ii) {
+              const uint32_t on = mask & (1u << ii);
+              sts_f32_if(av, v[ii], on);
+              sts_u16_if(ai, uint16_t(col0 + ii), on);
+              av += on ? 4u : 0u;
+              ai += on ? 2u : 0u;
+            }
+          } else {
+            int pos = pos0;  // the row overflows its list: it goes to the exact path
 #pragma unroll
             for (int ii = 0; ii < 32; ++ii) {
               if ((mask >> ii) & 1u) {
