@@ -34,7 +34,10 @@ constexpr int kRecurThreads = 256;
 constexpr int kMaxBlockEntries = 8192;  // list entries per (head, block) in a plan
 constexpr int kEntryBits = 13;          // entry index within a block: < 2^13
 static_assert(kMaxBlockEntries <= (1 << kEntryBits), "entry index must fit its key field");
-constexpr int kBucketTarget = 16;       // mean plan records per bucket aimed for
+#ifndef SDM_BUCKET_TARGET
+#define SDM_BUCKET_TARGET 4
+#endif
+constexpr int kBucketTarget = SDM_BUCKET_TARGET;  // mean plan records per bucket aimed for
 constexpr int kStreamMin = 4;           // mean records per stream and block, at least
 constexpr size_t kChunkBudget = size_t(4) << 30;  // workspace bytes per time chunk
 #ifndef SDM_RECUR_GROUP_BYTES

@@ -103,7 +103,9 @@ constexpr int kSelHeadBytes = 2 * kSelBuckets * 4;
 //      order and the bucket kb that holds the k-th largest.
 //   3. The entries of buckets 0..kb are staged, grouped by bucket.
 //   4. An entry's rank is its bucket's start plus the number of staged entries
-//      of its bucket that precede it; ranks below k are final positions.
+//      of its bucket that precede it; ranks below k are final positions.  The
+//      lanes take the staged entries in turn, so the bucket walks scale with
+//      the staged count, not with the entries each lane held.
 // A bucket holds a few entries unless the keys crowd together, so the rank
 // loops are short.  Returns false, writing nothing, if more than `cap` entries
 // would be staged (the caller then takes another path).
@@ -164,15 +166,16 @@ __device__ __forceinline__ bool warp_bucket_topk(const uint32_t (&key)[PL],
     }
   }
   __syncwarp();
-#pragma unroll
-  for (int i = 0; i < PL; ++i) {
-    if (b[i] <= kb) {
-      const uint64_t me = (uint64_t(key[i]) << 32) | uint64_t(~row[i]);
-      const int bs = start[b[i]], be = cur[b[i]];
-      int rank = bs;
-      for (int j = bs; j < be; ++j) rank += stage[j] > me ? 1 : 0;
-      if (rank < k) out[rank] = make_uint2(__float_as_uint(ord2f(key[i])), row[i]);
-    }
+  // ranks, by staged position (at most ceil(cap / 32) per lane), so that the
+  // warp walks only the buckets of staged entries
+  for (int q = lane; q < nst; q += 32) {
+    const uint64_t me = stage[q];
+    const uint32_t mk = uint32_t(me >> 32);
+    const int bq = int((hi - mk) >> sh);
+    const int bs = start[bq], be = cur[bq];
+    int rank = bs;
+    for (int j = bs; j < be; ++j) rank += stage[j] > me ? 1 : 0;
+    if (rank < k) out[rank] = make_uint2(__float_as_uint(ord2f(mk)), ~uint32_t(me));
   }
   return true;
 }
