@@ -209,6 +209,7 @@ __device__ inline uint32_t warp_select32(const uint32_t* cand, int n, int r, uin
 // Merge of one (step, side): sorted half lists (first k entries of each
 // survivor list) -> the n_sel selected slots and their softmax weights.
 // Selection order is unspecified unless `sorted` is set (then rank order).
+// With sv1 == sv2 == nullptr the lists are already in h1, h2.
 __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const uint2* sv2, int c2,
                           int n_sel, const uint32_t* stair, int n_stair, const uint32_t* front,
                           int nf, const int* ediv, uint64_t* h1, uint64_t* h2, uint32_t* cand, uint32_t* cell,
@@ -221,10 +222,12 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
     __syncwarp();
     return;
   }
-  for (int i = lane; i < p.k; i += 32) {
-    const uint2 a = sv1[i], b = sv2[i];
-    h1[i] = (uint64_t(a.x) << 32) | a.y;
-    h2[i] = (uint64_t(b.x) << 32) | b.y;
+  if (sv1 != nullptr) {  // else the caller has staged the lists in h1, h2
+    for (int i = lane; i < p.k; i += 32) {
+      const uint2 a = sv1[i], b = sv2[i];
+      h1[i] = (uint64_t(a.x) << 32) | a.y;
+      h2[i] = (uint64_t(b.x) << 32) | b.y;
+    }
   }
   __syncwarp();
   const uint32_t n = uint32_t(p.n);

@@ -58,7 +58,11 @@ size_t plan_smem_bytes(const Plan& p) { return plan_layout(p).total; }
 // ------------------------------------------------------------------ kernels
 // One CTA per (head, kMergeSteps steps); one warp per (step, side).  Writes
 // the W write and R read (slot, weight) pairs of each step to the lists
-// (row = bh * list_T + list_t0 + step), in rank order when `sorted`.
+// (row = bh * list_T + list_t0 + step), in rank order when `sorted`.  A warp
+// loads the half lists of its next (step, side) into registers (KPL entries
+// per lane, k <= 32 KPL) while it merges the current one; KPL = 0 leaves the
+// loads to merge_one.
+template <int KPL>
 __global__ void __launch_bounds__(kMergeWarps * 32)
 k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -85,15 +89,54 @@ k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   uint32_t* cell = cand + L.Sc;
   uint32_t* alt = cell + L.Sc;
   int* hist = reinterpret_cast<int*>(alt + 2 * L.Sc);
+  auto task_hr = [&](int pi) { return (size_t(bh) * p.Tc + s0 + (pi >> 1)) * 4 + (pi & 1) * 2; };
+  uint2 pa[KPL > 0 ? KPL : 1], pb[KPL > 0 ? KPL : 1];
+  int pc1 = 0, pc2 = 0;
+  auto prefetch = [&](int pi) {
+    const size_t hr = task_hr(pi);
+    pc1 = io.surv_cnt[hr];
+    pc2 = io.surv_cnt[hr + 1];
+    const uint2* l1 = io.surv + hr * p.C;
+    const uint2* l2 = l1 + p.C;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const int i = j * 32 + lane;
+      if (i < p.k) {
+        pa[j] = l1[i];
+        pb[j] = l2[i];
+      }
+    }
+  };
+  if (KPL > 0 && warp < 2 * np) prefetch(warp);
   for (int pi = warp; pi < 2 * np; pi += kMergeWarps) {
     const int tc = s0 + (pi >> 1), side = pi & 1;
-    const size_t hr = (size_t(bh) * p.Tc + tc) * 4 + side * 2;
+    const size_t hr = task_hr(pi);
     const int n_sel = side ? p.R : p.W;
     const size_t row = size_t(bh) * io.list_T + io.list_t0 + tc;
     float* w_out = (side ? io.out_wr : io.out_ww) + row * n_sel;
     uint32_t* s_out = reinterpret_cast<uint32_t*>(side ? io.out_ir : io.out_iw) + row * n_sel;
-    merge_one(p, io.surv + hr * p.C, io.surv_cnt[hr], io.surv + (hr + 1) * p.C,
-              io.surv_cnt[hr + 1], n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
+    const uint2* l1 = nullptr;
+    const uint2* l2 = nullptr;
+    int c1, c2;
+    if (KPL > 0) {
+#pragma unroll
+      for (int j = 0; j < KPL; ++j) {
+        const int i = j * 32 + lane;
+        if (i < p.k) {
+          h1[i] = (uint64_t(pa[j].x) << 32) | pa[j].y;
+          h2[i] = (uint64_t(pb[j].x) << 32) | pb[j].y;
+        }
+      }
+      c1 = pc1;
+      c2 = pc2;
+      if (pi + kMergeWarps < 2 * np) prefetch(pi + kMergeWarps);
+    } else {
+      l1 = io.surv + hr * p.C;
+      l2 = l1 + p.C;
+      c1 = io.surv_cnt[hr];
+      c2 = io.surv_cnt[hr + 1];
+    }
+    merge_one(p, l1, c1, l2, c2, n_sel, side ? stairR : stairW, side ? p.ncR : p.ncW,
               side ? frontR : frontW, side ? p.nfR : p.nfW, side ? edivR : edivW, h1, h2, cand,
               cell, alt, hist, sel,
               io.sorted != 0, w_out, s_out, st, int(hr), p.rule == 1 && side == 0);
@@ -151,10 +194,12 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    // exclusive scan of the bucket counts, one warp
-    const int per = (p.NB + 31) / 32;
-    const int g0 = min(p.NB, lane * per), g1 = min(p.NB, g0 + per);
+  {
+    // exclusive scan of the bucket counts over the whole CTA: each thread sums
+    // a run of buckets, a warp scan and a scan of the warp totals give its base
+    __shared__ int wtot[kPlanThreads / 32];
+    const int per = (p.NB + stride - 1) / stride;
+    const int g0 = min(p.NB, tid * per), g1 = min(p.NB, g0 + per);
     int sum = 0;
     for (int g = g0; g < g1; ++g) sum += start[g];
     int inc = sum;
@@ -163,14 +208,27 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
       const int y = __shfl_up_sync(0xffffffffu, inc, o);
       if (lane >= o) inc += y;
     }
-    int run = inc - sum;
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+      const int x = lane < kPlanThreads / 32 ? wtot[lane] : 0;
+      int wi = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += y;
+      }
+      if (lane < kPlanThreads / 32) wtot[lane] = wi - x;  // exclusive
+      if (lane == 31) start[p.NB] = wi;                   // all entries in range
+    }
+    __syncthreads();
+    int run = wtot[warp] + inc - sum;
     for (int g = g0; g < g1; ++g) {
       const int c = start[g];
       start[g] = run;
       cur[g] = run;
       run += c;
     }
-    if (lane == 31) start[p.NB] = inc;
   }
   __syncthreads();
   int* roff = io.roff + (size_t(bh) * p.nblk + blk) * (p.NB + 1);
@@ -273,15 +331,24 @@ k_plan(Plan p, PlanIO io, int t0, int tlen, DevStatus* st) {
   }
 }
 
+template <int KPL>
+static cudaError_t launch_merge_t(const Plan& p, const MergeIO& io, int t0, int tlen,
+                                  DevStatus* st, size_t smem, dim3 grid, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(k_merge<KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  k_merge<KPL><<<grid, kMergeWarps * 32, smem, s>>>(p, io, t0, tlen, st);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_merge(const Plan& p, const MergeIO& io, int t0, int tlen, DevStatus* st,
                          cudaStream_t s) {
   const size_t smem = merge_smem_bytes(p, kMergeWarps);
-  cudaError_t e = cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
-  if (e != cudaSuccess) return e;
   dim3 grid((tlen + kMergeSteps - 1) / kMergeSteps, p.BH);
-  k_merge<<<grid, kMergeWarps * 32, smem, s>>>(p, io, t0, tlen, st);
-  return cudaGetLastError();
+  if (p.k <= 32) return launch_merge_t<1>(p, io, t0, tlen, st, smem, grid, s);
+  if (p.k <= 64) return launch_merge_t<2>(p, io, t0, tlen, st, smem, grid, s);
+  if (p.k <= 128) return launch_merge_t<4>(p, io, t0, tlen, st, smem, grid, s);
+  return launch_merge_t<0>(p, io, t0, tlen, st, smem, grid, s);
 }
 
 cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevStatus* st,

@@ -373,7 +373,7 @@ k_score_tc(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUten
     const int ew = warp - 2;
     const int K2 = next_pow2(k < 2 ? 2 : k);
     unsigned char* wscr = smem + L.sel + size_t(ew) * size_t(kSelHeadBytes + 8 * L.cap);
-    int* scr = reinterpret_cast<int*>(wscr);
+    uint32_t* scr = reinterpret_cast<uint32_t*>(wscr);
     uint64_t* stage = reinterpret_cast<uint64_t*>(wscr + kSelHeadBytes);
     const bool keep_all = !(a.z > -1e30f);
     const int nstat = ntiles < 2 ? ntiles : 2;

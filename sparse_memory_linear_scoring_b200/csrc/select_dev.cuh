@@ -89,16 +89,22 @@ __device__ __forceinline__ void warp_gather_topk(const uint32_t (&key)[PL],
   }
 }
 
-// Scratch of warp_bucket_topk per warp: kSelBuckets cursors, kSelBuckets
-// bucket starts, then the staged 64-bit keys.
-constexpr int kSelBuckets = 64;
-constexpr int kSelHeadBytes = 2 * kSelBuckets * 4;
+// Scratch of warp_bucket_topk per warp: kSelBuckets words (bucket start << 16
+// | cursor), then the staged 64-bit keys.
+#ifndef SDM_SEL_BUCKETS
+#define SDM_SEL_BUCKETS 128
+#endif
+constexpr int kSelBuckets = SDM_SEL_BUCKETS;
+static_assert(kSelBuckets == 64 || kSelBuckets == 128 || kSelBuckets == 256,
+              "64, 128 or 256 buckets");
+constexpr int kSelHeadBytes = kSelBuckets * 4;
 
 // The k best of the c valid (key, row) entries held PL per lane (entry i*32 + l
-// in lane l; 1 <= k <= c; rows distinct), written to out[0..k) in (key desc,
-// row asc) order as (value bits, row) pairs, value = ord2f(key).
-//   1. The keys are counted into 64 buckets of the key range, bucket 0 holding
-//      the largest (bucket = (max - key) >> shift, monotone in the key).
+// in lane l; 1 <= k <= c <= 65535; rows distinct), written to out[0..k) in (key
+// desc, row asc) order as (value bits, row) pairs, value = ord2f(key).
+//   1. The keys are counted into kSelBuckets buckets of the key range, bucket 0
+//      holding the largest (bucket = (max - key) >> shift, monotone in the
+//      key); each lane owns kSelBuckets / 32 consecutive buckets.
 //   2. A warp scan of the counts gives every bucket's start in the output
 //      order and the bucket kb that holds the k-th largest.
 //   3. The entries of buckets 0..kb are staged, grouped by bucket.
@@ -112,10 +118,11 @@ constexpr int kSelHeadBytes = 2 * kSelBuckets * 4;
 template <int PL>
 __device__ __forceinline__ bool warp_bucket_topk(const uint32_t (&key)[PL],
                                                  const uint32_t (&row)[PL], int c, int k,
-                                                 int* scr, uint64_t* stage, int cap, uint2* out) {
+                                                 uint32_t* bkt, uint64_t* stage, int cap,
+                                                 uint2* out) {
+  constexpr int BPL = kSelBuckets / 32;  // buckets per lane
+  constexpr int LOGB = kSelBuckets == 64 ? 6 : (kSelBuckets == 128 ? 7 : 8);
   const int lane = threadIdx.x & 31;
-  int* cur = scr;                 // [64] counts, then cursors
-  int* start = scr + kSelBuckets; // [64] bucket starts
   uint32_t lo = 0xffffffffu, hi = 0u;
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
@@ -126,42 +133,59 @@ __device__ __forceinline__ bool warp_bucket_topk(const uint32_t (&key)[PL],
   }
   lo = __reduce_min_sync(0xffffffffu, lo);
   hi = __reduce_max_sync(0xffffffffu, hi);
-  const uint32_t span = hi - lo;
-  const int nbits = 32 - __clz(span);  // span < 2^nbits
-  const int sh = nbits > 6 ? nbits - 6 : 0;
-  cur[lane] = 0;
-  cur[lane + 32] = 0;
+  const int nbits = 32 - __clz(hi - lo);  // hi - lo < 2^nbits
+  const int sh = nbits > LOGB ? nbits - LOGB : 0;
+  uint32_t* mine = bkt + lane * BPL;
+#pragma unroll
+  for (int j = 0; j < BPL; ++j) mine[j] = 0u;
   __syncwarp();
   int b[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     b[i] = i * 32 + lane < c ? int((hi - key[i]) >> sh) : kSelBuckets;
-    if (b[i] < kSelBuckets) atomicAdd(&cur[b[i]], 1);
+    if (b[i] < kSelBuckets) atomicAdd(&bkt[b[i]], 1u);
   }
   __syncwarp();
-  const int c0 = cur[2 * lane], c1 = cur[2 * lane + 1];
-  int incl = c0 + c1;
+  // the lane's buckets: counts and running sums, then the warp scan of the totals
+  int cnt[BPL], run[BPL];
+  int tot = 0;
+#pragma unroll
+  for (int j = 0; j < BPL; ++j) {
+    cnt[j] = int(mine[j]);
+    tot += cnt[j];
+    run[j] = tot;
+  }
+  int incl = tot;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, incl, d);
     if (lane >= d) incl += y;
   }
-  const int s0 = incl - c0 - c1, s1 = s0 + c0;  // starts of buckets 2 lane, 2 lane + 1
-  const unsigned ge = __ballot_sync(0xffffffffu, incl >= k);  // lane 31 holds c >= k
-  const int lk = __ffs(ge) - 1;
-  const int kb = 2 * lk + __shfl_sync(0xffffffffu, s1 >= k ? 0 : 1, lk);
-  const int nst = __shfl_sync(0xffffffffu, (kb & 1) ? incl : s1, kb >> 1);  // end of bucket kb
+  const int excl = incl - tot;
+  // kb: the first bucket whose end reaches k (lane 31's last end is c >= k)
+  int myj = BPL, myend = 0;
+#pragma unroll
+  for (int j = BPL - 1; j >= 0; --j) {
+    if (excl + run[j] >= k) {
+      myj = j;
+      myend = excl + run[j];
+    }
+  }
+  const int lk = __ffs(__ballot_sync(0xffffffffu, myj < BPL)) - 1;
+  const int kb = lk * BPL + __shfl_sync(0xffffffffu, myj, lk);
+  const int nst = __shfl_sync(0xffffffffu, myend, lk);  // end of bucket kb
   if (nst > cap) return false;
   __syncwarp();
-  cur[2 * lane] = s0;
-  cur[2 * lane + 1] = s1;
-  start[2 * lane] = s0;
-  start[2 * lane + 1] = s1;
+#pragma unroll
+  for (int j = 0; j < BPL; ++j) {
+    const uint32_t st = uint32_t(excl + run[j] - cnt[j]);
+    mine[j] = (st << 16) | st;  // start, cursor
+  }
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     if (b[i] <= kb) {
-      const int pos = atomicAdd(&cur[b[i]], 1);
+      const int pos = int(atomicAdd(&bkt[b[i]], 1u) & 0xffffu);
       stage[pos] = (uint64_t(key[i]) << 32) | uint64_t(~row[i]);
     }
   }
@@ -171,8 +195,8 @@ __device__ __forceinline__ bool warp_bucket_topk(const uint32_t (&key)[PL],
   for (int q = lane; q < nst; q += 32) {
     const uint64_t me = stage[q];
     const uint32_t mk = uint32_t(me >> 32);
-    const int bq = int((hi - mk) >> sh);
-    const int bs = start[bq], be = cur[bq];
+    const uint32_t w = bkt[(hi - mk) >> sh];
+    const int bs = int(w >> 16), be = int(w & 0xffffu);
     int rank = bs;
     for (int j = bs; j < be; ++j) rank += stage[j] > me ? 1 : 0;
     if (rank < k) out[rank] = make_uint2(__float_as_uint(ord2f(mk)), ~uint32_t(me));

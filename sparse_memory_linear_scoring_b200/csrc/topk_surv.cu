@@ -26,7 +26,7 @@ k_topk_surv(Plan p, int tlen, int* __restrict__ cnt, uint2* __restrict__ surv, D
   const int K2 = next_pow2(p.k < 2 ? 2 : p.k);
   const int cap = p.C > K2 ? p.C : K2;
   unsigned char* wscr = smem + size_t(warp) * (kSelHeadBytes + 8 * size_t(cap));
-  int* scr = reinterpret_cast<int*>(wscr);
+  uint32_t* scr = reinterpret_cast<uint32_t*>(wscr);
   uint64_t* sel = reinterpret_cast<uint64_t*>(wscr + kSelHeadBytes);
   const int nrows = p.BH * tlen * 4;
   for (int w = blockIdx.x * kTopkWarps + warp; w < nrows; w += gridDim.x * kTopkWarps) {
