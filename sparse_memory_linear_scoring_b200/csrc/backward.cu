@@ -85,6 +85,18 @@ __global__ void k_bwd_init(const float4* __restrict__ M0, float4* __restrict__ M
 template <typename Tv>
 __device__ __forceinline__ float ldv(const Tv* p) { return to_f32(__ldg(p)); }
 
+// two consecutive elements (the first at an even index) as float
+__device__ __forceinline__ void ld2(const float* p, float& a, float& b) {
+  const float2 v = __ldg(reinterpret_cast<const float2*>(p));
+  a = v.x;
+  b = v.y;
+}
+__device__ __forceinline__ void ld2(const __nv_bfloat16* p, float& a, float& b) {
+  const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+  a = __uint_as_float(u << 16);
+  b = __uint_as_float(u & 0xffff0000u);
+}
+
 // One stream (LPR lanes, F floats of a row each) per group of buckets, as in
 // the forward recurrence; records backward.
 template <typename Tv, int LPR, int F>
@@ -237,32 +249,48 @@ k_sel_bwd(Plan p, const Tin* __restrict__ q, const Tin* __restrict__ k,
         rows[j] = int(half ? slot % uint32_t(p.n) : slot / uint32_t(p.n));
       }
       __syncwarp();
-      // dx_h = sum_j ds_j C_h[row_j]
-      for (int c = lane; c < p.dh; c += 32) {
-        float acc = 0.f;
-        for (int j = 0; j < n_sel; ++j) acc = fmaf(ds[j], to_f32(C[size_t(rows[j]) * p.dh + c]), acc);
-        dx[half * p.dh + c] = acc;
+      // dx_h = sum_j ds_j C_h[row_j] (two columns per lane when d_h is even)
+      if ((p.dh & 1) == 0) {
+        for (int c = 2 * lane; c < p.dh; c += 64) {
+          float a0 = 0.f, a1 = 0.f;
+          for (int j = 0; j < n_sel; ++j) {
+            float c0, c1;
+            ld2(C + size_t(rows[j]) * p.dh + c, c0, c1);
+            a0 = fmaf(ds[j], c0, a0);
+            a1 = fmaf(ds[j], c1, a1);
+          }
+          dx[half * p.dh + c] = a0;
+          dx[half * p.dh + c + 1] = a1;
+        }
+      } else {
+        for (int c = lane; c < p.dh; c += 32) {
+          float acc = 0.f;
+          for (int j = 0; j < n_sel; ++j)
+            acc = fmaf(ds[j], to_f32(C[size_t(rows[j]) * p.dh + c]), acc);
+          dx[half * p.dh + c] = acc;
+        }
       }
-      // dC_h[row] += (sum of ds over the entries on that row) x_h: one update
-      // per distinct row (the first entry of each row collects the sum)
+      // dC_h[row] += (sum of ds over the entries on that row) x_h: within each
+      // group of 32 entries, one update per distinct row (its lowest lane sums
+      // the group's entries on that row)
       for (int j0 = 0; j0 < n_sel; j0 += 32) {
         const int j = j0 + lane;
-        bool lead = false;
+        const bool valid = j < n_sel;
+        const int rj = valid ? rows[j] : -1 - lane;
+        const unsigned peers = __match_any_sync(0xffffffffu, rj);
+        const bool lead = valid && __ffs(peers) - 1 == lane;
         float sum = 0.f;
-        if (j < n_sel) {
-          lead = true;
-          for (int i = 0; i < j; ++i) lead &= rows[i] != rows[j];
-          if (lead)
-            for (int i = j; i < n_sel; ++i) sum += rows[i] == rows[j] ? ds[i] : 0.f;
+        if (lead) {
+          for (unsigned m = peers; m; m &= m - 1) sum += ds[j0 + __ffs(m) - 1];
         }
         unsigned m = __ballot_sync(0xffffffffu, lead);
         while (m) {
           const int src = __ffs(m) - 1;
           m &= m - 1;
-          const int rj = __shfl_sync(0xffffffffu, j < n_sel ? rows[j] : 0, src);
+          const int rs = __shfl_sync(0xffffffffu, rj, src);
           const float sj = __shfl_sync(0xffffffffu, sum, src);
           for (int c = lane; c < p.dh; c += 32)
-            atomicAdd(dC + size_t(rj) * p.dh + c, sj * to_f32(x[half * p.dh + c]));
+            atomicAdd(dC + size_t(rs) * p.dh + c, sj * to_f32(x[half * p.dh + c]));
         }
       }
       __syncwarp();
