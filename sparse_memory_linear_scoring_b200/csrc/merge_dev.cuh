@@ -251,28 +251,40 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   hist[lane + 32] = 0;
   __syncwarp();
   int nc = 0;
-  for (int i0 = 0; i0 < n_stair; i0 += 32) {
-    const int i = i0 + lane;
-    uint32_t x = 0, ab = 0;
-    if (i < n_stair) {
-      ab = stair[i];
-      x = f2ord(hval(h1[ab & 0xffff]) + hval(h2[ab >> 16]));
+  // two groups of 32 cells per trip, their loads issued together
+  for (int i0 = 0; i0 < n_stair; i0 += 64) {
+    uint32_t x[2] = {0u, 0u}, ab[2] = {0u, 0u};
+    bool keep[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + 32 * u + lane;
+      if (i < n_stair) ab[u] = stair[i];
     }
-    const bool keep = i < n_stair && x >= lb;
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = nc + __popc(m & lanemask_lt());
-      cand[pos] = x;
-      cell[pos] = ab;
-      atomicAdd(&hist[(hi - x) >> sh], 1);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + 32 * u + lane;
+      if (i < n_stair) x[u] = f2ord(hval(h1[ab[u] & 0xffff]) + hval(h2[ab[u] >> 16]));
+      keep[u] = i < n_stair && x[u] >= lb;
     }
-    nc += __popc(m);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const unsigned m = __ballot_sync(0xffffffffu, keep[u]);
+      if (keep[u]) {
+        const int pos = nc + __popc(m & lanemask_lt());
+        cand[pos] = x[u];
+        cell[pos] = ab[u];
+        atomicAdd(&hist[(hi - x[u]) >> sh], 1);
+      }
+      nc += __popc(m);
+    }
   }
   __syncwarp();
   // the n_sel-th best: a warp scan of the bucket counts finds the bucket kb
   // that holds it and its rank r there; a bucket of at most 32 entries is
   // sorted across the warp, a larger one (crowded scores) goes to quickselect
   uint32_t vstar;
+  int n_gt = 0, n_eq = 0;  // candidates above / equal to vstar
+  bool counted = false;
   {
     const int c0 = hist[2 * lane], c1 = hist[2 * lane + 1];
     int incl = c0 + c1;
@@ -298,9 +310,15 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
         nb += __popc(m);
       }
       __syncwarp();
-      uint32_t y = lane < kb1 - kb0 ? alt[lane] : 0u;
+      const bool live = lane < kb1 - kb0;  // the sorted bucket fills lanes 0..m-1
+      uint32_t y = live ? alt[lane] : 0u;
       y = warp_sort32_desc_u32(y);
       vstar = __shfl_sync(0xffffffffu, y, n_sel - kb0 - 1);
+      // the buckets before kb hold only candidates above vstar, those after it
+      // only candidates below; in kb, count from the sorted values
+      n_gt = kb0 + __popc(__ballot_sync(0xffffffffu, live && y > vstar));
+      n_eq = __popc(__ballot_sync(0xffffffffu, live && y == vstar));
+      counted = true;
       __syncwarp();
     } else {
       vstar = warp_select32(cand, nc, n_sel, alt, alt + (nc + 31) / 32 * 32);
@@ -308,14 +326,15 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   }
   // exact when every candidate outside the staircase scores strictly below the
   // n_sel-th and no other candidate ties it
-  int n_gt = 0, n_eq = 0;
-  for (int i = lane; i < nc; i += 32) {
-    const uint32_t x = cand[i];
-    n_gt += x > vstar;
-    n_eq += x == vstar;
+  if (!counted) {
+    for (int i = lane; i < nc; i += 32) {
+      const uint32_t x = cand[i];
+      n_gt += x > vstar;
+      n_eq += x == vstar;
+    }
+    n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+    n_eq = __reduce_add_sync(0xffffffffu, n_eq);
   }
-  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
-  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
   bool bad = false;
   for (int i = lane; i < nf; i += 32) {
     const uint32_t ab = front[i];

@@ -61,9 +61,11 @@ size_t plan_smem_bytes(const Plan& p) { return plan_layout(p).total; }
 // (row = bh * list_T + list_t0 + step), in rank order when `sorted`.  A warp
 // loads the half lists of its next (step, side) into registers (KPL entries
 // per lane, k <= 32 KPL) while it merges the current one; KPL = 0 leaves the
-// loads to merge_one.
+// loads to merge_one.  The launch bounds keep the k <= 64 kernels at 64
+// registers (four CTAs per SM, the shared-memory limit too) and give the wider
+// ones room for their lists without spilling.
 template <int KPL>
-__global__ void __launch_bounds__(kMergeWarps * 32)
+__global__ void __launch_bounds__(kMergeWarps * 32, KPL >= 4 ? 3 : 4)
 k_merge(Plan p, MergeIO io, int t0, int tlen, DevStatus* st) {
   extern __shared__ __align__(16) unsigned char smem[];
   const MergeLayout L = merge_layout(p, kMergeWarps);
