@@ -178,6 +178,31 @@ def test_duplicate_codebook_rows(base):
     _check_forward(base, inp, ref)
 
 
+@pytest.mark.parametrize("base", [
+    config(2).with_(B=1, H=2, T=200, m0_sd=0.5),
+    config(3).with_(B=1, H=2, T=120, m0_sd=0.5),
+], ids=["bf16-tensor-core", "bf16-tensor-core-filter"])
+def test_outlier_codebook_row(base):
+    """One codebook row per half scaled by 64 (a power of two: exact in bf16), in a
+    column past the 512 the threshold statistics read: every token whose score
+    on row 0 is positive gets one score far above the rest.  The kept scores then
+    crowd into the lowest buckets of their key range, which sends the in-kernel
+    top-k to its bitwise-search path, gives the survivor top-k one large bucket,
+    and crowds the merge's candidate buckets (its quickselect path)."""
+    import sparse_memory_linear_scoring_b200 as s
+    mode = s.query_plan(s.make_dims(**base.dims()))["scoring_mode"]
+    assert mode == (1 if base.d_qk == 128 else 2)
+    inp = gen_inputs(base)
+    j = base.n_sub - 3
+    assert j >= 512
+    for name in ("C1", "C2"):
+        c = inp[name].clone()
+        c[:, j] = c[:, 0] * 64
+        inp[name] = c
+    ref = oracle_full(inp, base, lists=True)
+    _check_forward(base, inp, ref)
+
+
 def test_fp32_wide_rows():
     cfg = config(0).with_(B=2, H=3, T=200, d_v=128, d_qk=24, n_sub=16, k=6, W=20, R=12,
                           m0_sd=1.0)
