@@ -264,7 +264,9 @@ SDM_API const char* sdm_status_string(int status);
  * segments backward in reverse order, each given the table at its start and
  * the dM0 of the segment after it as its dM_T); the workspace
  * (sdm_backward_workspace_bytes) holds the plan and the row each access of the
- * forward saw, (2W + R) d_v floats per token-head, plus a working copy of M0.
+ * forward saw, (2W + R) d_v floats per token-head, plus a working table the
+ * size of M0 (rows are read from M0 until first written there; M0 is not
+ * copied) and one byte per slot marking the rows written.
  * The codebook gradients are accumulated with float atomics, so their last
  * bits vary from call to call.  Same pointer, stream and error conventions as
  * sdm_forward (dalpha, dbeta: 4-byte alignment).

@@ -21,9 +21,10 @@
 //    dx_h = sum_j ds_h[j] C_h[j] (into dk' or dq') and dC_h[j] += ds_h[j] x_h.
 //
 // The reverse recurrence needs the row values the forward saw (m, M_t[slot]).
-// They are recomputed: the forward recurrence runs again from M_0 on a working
-// copy, in the mode that stores, per record, the row it finds (launch_recur with
-// snap).  The plan's records already sort every slot's accesses by time inside
+// They are recomputed: the forward recurrence runs again from M_0, in the mode
+// that stores, per record, the row it finds (launch_recur with snap); it reads
+// a row from M_0 until it first writes the row into its working table, so M_0
+// is never copied.  The plan's records already sort every slot's accesses by time inside
 // a block, so the reverse kernel walks the same per-slot streams: blocks from
 // last to first, each block's records from last to first, carrying g between
 // blocks in dM_0's row.
@@ -36,7 +37,8 @@ namespace sdm {
 constexpr int kBwdThreads = 256;
 
 struct BwdLayout {
-  size_t off_status, off_rec, off_roff, off_rent, off_snap, off_g, off_ga, off_mw, total;
+  size_t off_status, off_rec, off_roff, off_rent, off_snap, off_g, off_ga, off_mw, off_touch,
+      total;
 };
 
 static BwdLayout bwd_layout(const Plan& p) {
@@ -53,6 +55,7 @@ static BwdLayout bwd_layout(const Plan& p) {
   L.off_g = o; o = al(o + ents * 4);
   L.off_ga = o; o = al(o + ents * 4);
   L.off_mw = o; o = al(o + size_t(p.BH) * size_t(p.N) * p.dv * 4);
+  L.off_touch = o; o = al(o + size_t(p.BH) * size_t(p.N));
   L.total = o;
   return L;
 }
@@ -65,16 +68,13 @@ static int bwd_plan(const sdm_dims* d, Plan* p) {
   return SDM_OK;
 }
 
-__global__ void k_bwd_init(const float4* __restrict__ M0, float4* __restrict__ Mw,
-                           const float4* __restrict__ dMT, float4* __restrict__ dM0,
+__global__ void k_bwd_init(const float4* __restrict__ dMT, float4* __restrict__ dM0,
                            size_t n4, float4* __restrict__ dv, size_t nv4,
                            float4* __restrict__ dC1, float4* __restrict__ dC2, size_t nc4) {
   const size_t stride = size_t(gridDim.x) * blockDim.x;
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    Mw[i] = M0[i];
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride)
     dM0[i] = dMT ? dMT[i] : z;
-  }
   for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nv4; i += stride) dv[i] = z;
   for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nc4; i += stride) {
     dC1[i] = z;
@@ -374,14 +374,16 @@ extern "C" int sdm_backward(const void* q, const void* k, const void* v, const f
   float* gent = reinterpret_cast<float*>(w + L.off_g);
   float* gal = reinterpret_cast<float*>(w + L.off_ga);
   float* Mw = reinterpret_cast<float*>(w + L.off_mw);
+  uint8_t* touched = reinterpret_cast<uint8_t*>(w + L.off_touch);
   if (launch_init(p, st, s) != cudaSuccess) return SDM_ERR_CUDA;
-  // working copy of M_0, dM_0 = dM_T (or 0), dv = dC = 0
+  // dM_0 = dM_T (or 0), dv = dC = 0, no row of the working table written yet
+  if (cudaMemsetAsync(touched, 0, size_t(p.BH) * size_t(p.N), s) != cudaSuccess)
+    return SDM_ERR_CUDA;
   {
     const size_t n4 = size_t(p.BH) * size_t(p.N) * p.dv / 4;
     const size_t nv4 = size_t(p.BH) * p.T * p.dv / 4;
     const size_t nc4 = size_t(p.H) * p.n * p.dh / 4;
     k_bwd_init<<<148 * 8, 256, 0, s>>>(
-        reinterpret_cast<const float4*>(M0), reinterpret_cast<float4*>(Mw),
         reinterpret_cast<const float4*>(dM_T), reinterpret_cast<float4*>(dM0), n4,
         reinterpret_cast<float4*>(dv), nv4, reinterpret_cast<float4*>(dC1),
         reinterpret_cast<float4*>(dC2), p.dh % 4 == 0 ? nc4 : 0);
@@ -407,7 +409,8 @@ extern "C" int sdm_backward(const void* q, const void* k, const void* v, const f
   pio.rent = rent;
   if (launch_plan(p, pio, 0, p.T, st, s) != cudaSuccess) return SDM_ERR_CUDA;
   // the forward recurrence again from M_0, saving the rows each record sees
-  if (launch_recur(p, v, Mw, nullptr, rec, roff, 0, p.T, s, snap) != cudaSuccess)
+  if (launch_recur(p, v, Mw, nullptr, rec, roff, 0, p.T, s,
+                   SaveIO{snap, static_cast<const float*>(M0), touched}) != cudaSuccess)
     return SDM_ERR_CUDA;
   // reverse recurrence
   cudaError_t e = p.dtype == SDM_DTYPE_F32

@@ -195,7 +195,7 @@ template <typename Tv, int LPR, int F, bool SAVE>
 __global__ void __launch_bounds__(kRecurThreads, kRecurWarps / 148 / (kRecurThreads / 32))
 k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restrict__ o,
         const int4* __restrict__ rec, const int* __restrict__ roff, int t0, int tlen, int bh0,
-        int nbh, float* __restrict__ snap) {
+        int nbh, SaveIO sv) {
   using SM = RecurSmem<Tv, LPR, F>;
   constexpr int dv = LPR * F;
   constexpr int U = SM::U;
@@ -215,6 +215,9 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
   const int nb = (tlen + p.P - 1) / p.P;
   const int g0 = s * p.mb, g1 = g0 + p.mb;
   float* Mh = M + size_t(bh) * size_t(p.N) * dv + sl * F;
+  // snapshot mode: rows not yet stored by this walk come from M0
+  const float* M0h = SAVE ? sv.M0 + size_t(bh) * size_t(p.N) * dv + sl * F : nullptr;
+  uint8_t* toh = SAVE ? sv.touched + size_t(bh) * size_t(p.N) : nullptr;
   const size_t trow = size_t(bh) * p.T + t0;
   const Tv* vh = v + trow * dv + sl * F;
   float* oh = o + trow * dv + sl * F;
@@ -321,6 +324,16 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
     // visible.
     uint32_t head = 0, last = 0;  // per record: first / last of its slot run
     VRaw<Tv, F> vr[SM::kVReg ? U : 1];
+    // snapshot mode: which records' rows the walk has already written (bit u),
+    // all flags loaded before the copies that depend on them
+    uint32_t written = 0;
+    if constexpr (SAVE) {
+      uint8_t fl[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) fl[u] = u < n ? toh[unsigned(lds2(&rs[u]).x)] : uint8_t(0);
+#pragma unroll
+      for (int u = 0; u < U; ++u) written |= uint32_t(fl[u] != 0) << u;
+    }
     {
       int prev = -1;
 #pragma unroll
@@ -330,7 +343,11 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
         if (u == 0 || u == t1 || sm.x != prev) {
           head |= 1u << u;
           if (u > 0) last |= 1u << (u - 1);
-          cp_bytes<F * 4>(mrow + u * dv, Mh + size_t(unsigned(sm.x)) * dv);
+          const float* src = Mh + size_t(unsigned(sm.x)) * dv;
+          if constexpr (SAVE) {
+            if (!((written >> u) & 1u)) src = M0h + size_t(unsigned(sm.x)) * dv;
+          }
+          cp_bytes<F * 4>(mrow + u * dv, src);
         }
         if (!(sm.y & 1)) {
           if constexpr (SM::kVReg)
@@ -363,7 +380,7 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
           // the row as this record finds it (record index as in rec)
           const size_t ri = u < t1 ? (size_t(bh) * p.nblk + b) * p.E + pos + u
                                    : (size_t(bh) * p.nblk + b + 1) * p.E + npos + (u - t1);
-          st_row<F>(snap + ri * dv + sl * F, cur);
+          st_row<F>(sv.snap + ri * dv + sl * F, cur);
         }
         if (!(r.y & 1)) {
 #pragma unroll
@@ -378,7 +395,10 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
           red_row<F>(oh + size_t(r.y >> 1) * dv, cur, f1);
         }
         if ((last >> u) & 1u) {
-          if (dirty) st_row<F>(Mh + size_t(unsigned(r.x)) * dv, cur);
+          if (dirty) {
+            st_row<F>(Mh + size_t(unsigned(r.x)) * dv, cur);
+            if constexpr (SAVE) toh[unsigned(r.x)] = 1;  // every lane: its own later loads see it
+          }
           dirty = false;
         }
       }
@@ -409,7 +429,7 @@ k_recur(Plan p, const Tv* __restrict__ v, float* __restrict__ M, float* __restri
 template <typename Tv, int LPR, int F, bool SAVE>
 static cudaError_t launch_recur_t(const Plan& p, const void* v, float* M, float* o,
                                   const int4* rec, const int* roff, int t0, int tlen,
-                                  cudaStream_t s, float* snap) {
+                                  cudaStream_t s, SaveIO sv) {
   const size_t smem = RecurSmem<Tv, LPR, F>::total;
   cudaError_t e = cudaFuncSetAttribute(k_recur<Tv, LPR, F, SAVE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -421,7 +441,7 @@ static cudaError_t launch_recur_t(const Plan& p, const void* v, float* M, float*
     const long long threads = (long long)nbh * p.S * LPR;
     const int grid = int((threads + kRecurThreads - 1) / kRecurThreads);
     k_recur<Tv, LPR, F, SAVE><<<grid, kRecurThreads, smem, s>>>(
-        p, (const Tv*)v, M, o, rec, roff, t0, tlen, bh0, nbh, snap);
+        p, (const Tv*)v, M, o, rec, roff, t0, tlen, bh0, nbh, sv);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -440,32 +460,33 @@ int recur_lanes_per_row(int dv) { return dv / recur_floats_per_lane(dv); }
 template <typename Tv, int DV>
 static cudaError_t launch_recur_w(const Plan& p, const void* v, float* M, float* o,
                                   const int4* rec, const int* roff, int t0, int tlen,
-                                  cudaStream_t s, float* snap) {
+                                  cudaStream_t s, SaveIO sv) {
   constexpr int F = recur_floats_per_lane(DV);
-  if (snap) return launch_recur_t<Tv, DV / F, F, true>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-  return launch_recur_t<Tv, DV / F, F, false>(p, v, M, o, rec, roff, t0, tlen, s, nullptr);
+  if (sv.snap) return launch_recur_t<Tv, DV / F, F, true>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+  return launch_recur_t<Tv, DV / F, F, false>(p, v, M, o, rec, roff, t0, tlen, s,
+                                               SaveIO{nullptr, nullptr, nullptr});
 }
 
 template <typename Tv>
 static cudaError_t launch_recur_dt(const Plan& p, const void* v, float* M, float* o,
                                    const int4* rec, const int* roff, int t0, int tlen,
-                                   cudaStream_t s, float* snap) {
+                                   cudaStream_t s, SaveIO sv) {
   switch (p.dv) {
-    case 4: return launch_recur_w<Tv, 4>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-    case 8: return launch_recur_w<Tv, 8>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-    case 16: return launch_recur_w<Tv, 16>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-    case 32: return launch_recur_w<Tv, 32>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-    case 64: return launch_recur_w<Tv, 64>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-    case 128: return launch_recur_w<Tv, 128>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    case 4: return launch_recur_w<Tv, 4>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+    case 8: return launch_recur_w<Tv, 8>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+    case 16: return launch_recur_w<Tv, 16>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+    case 32: return launch_recur_w<Tv, 32>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+    case 64: return launch_recur_w<Tv, 64>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+    case 128: return launch_recur_w<Tv, 128>(p, v, M, o, rec, roff, t0, tlen, s, sv);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_recur(const Plan& p, const void* v, float* M, float* o, const int4* rec,
-                         const int* roff, int t0, int tlen, cudaStream_t s, float* snap) {
+                         const int* roff, int t0, int tlen, cudaStream_t s, SaveIO sv) {
   if (p.dtype == SDM_DTYPE_F32)
-    return launch_recur_dt<float>(p, v, M, o, rec, roff, t0, tlen, s, snap);
-  return launch_recur_dt<__nv_bfloat16>(p, v, M, o, rec, roff, t0, tlen, s, snap);
+    return launch_recur_dt<float>(p, v, M, o, rec, roff, t0, tlen, s, sv);
+  return launch_recur_dt<__nv_bfloat16>(p, v, M, o, rec, roff, t0, tlen, s, sv);
 }
 
 }  // namespace sdm

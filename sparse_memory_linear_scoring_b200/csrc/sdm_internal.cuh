@@ -209,11 +209,18 @@ cudaError_t launch_plan(const Plan& p, const PlanIO& io, int t0, int tlen, DevSt
                         cudaStream_t s);
 
 // snap == nullptr: the recurrence (writes into M, reads added into o).  snap
-// given: the same walk over M, with no o, storing at every record the row it
-// sees before the record's effect (snap[record] = d_v floats, record index as
-// in rec) -- the values the backward pass needs.
+// given: the same walk, with no o, storing at every record the row it sees
+// before the record's effect (snap[record] = d_v floats, record index as in rec)
+// -- the values the backward pass needs; it starts from the table M0 without
+// copying it: a row is read from M0 until the walk first stores it into M,
+// which it records in touched (one byte per slot and head, zero at the start).
+struct SaveIO {
+  float* snap;
+  const float* M0;
+  uint8_t* touched;
+};
 cudaError_t launch_recur(const Plan& p, const void* v, float* M, float* o, const int4* rec,
                          const int* roff, int t0, int tlen, cudaStream_t s,
-                         float* snap = nullptr);
+                         SaveIO sv = SaveIO{nullptr, nullptr, nullptr});
 
 }  // namespace sdm
