@@ -82,10 +82,10 @@ def peaks():
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one k_recur
 # launch per token-head, measured by ncu on the pages-scale workload at
-# T = 1024 (8192 token-heads): 271.0 MB read + 90.2 MB written.  Valid only for
+# T = 1024 (8192 token-heads): 271.6 MB read + 90.4 MB written.  Valid only for
 # the recurrence source it was taken on (its SHA-256 below).
-RECUR_DRAM_BYTES_PER_TOKEN_HEAD = (270994944 + 90222848) / 8192.0
-RECUR_DRAM_SOURCE_SHA256 = "3a122f63b19354f79f7c120d12c32d7e52a7672ad3f17db88e3932bd6c7b5fb1"
+RECUR_DRAM_BYTES_PER_TOKEN_HEAD = (271587584 + 90435072) / 8192.0
+RECUR_DRAM_SOURCE_SHA256 = "0ee48857b052a60d68bbc1fd1273470b53448c57b4d0531cd578677d51ee9fc9"
 
 
 def recur_traffic(token_heads: int):

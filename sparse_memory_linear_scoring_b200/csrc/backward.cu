@@ -303,7 +303,11 @@ static cudaError_t launch_bwd_w(const Plan& p, const void* v, const float* alpha
                                 const float* d_o, float* dv, float* dM, const int4* rec,
                                 const int* roff, const int* rent, const float* snap, float* gent,
                                 float* gal, cudaStream_t s) {
-  constexpr int F = DV / 32 >= 1 ? (DV / 32 > 8 ? 8 : DV / 32) : 1;
+#ifndef SDM_BWD_LANE_FLOATS
+#define SDM_BWD_LANE_FLOATS 2  // floats per lane = this x d_v / 32: two streams per warp at d_v = 64
+#endif
+  constexpr int F0 = SDM_BWD_LANE_FLOATS * DV / 32;
+  constexpr int F = F0 >= 1 ? (F0 > 8 ? 8 : F0) : 1;
   constexpr int LPR = DV / F;
   static_assert(LPR <= 32 && (32 % LPR) == 0, "lanes per row");
   const long long threads = (long long)p.BH * p.S * LPR;
