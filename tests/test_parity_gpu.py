@@ -203,6 +203,24 @@ def test_outlier_codebook_row(base):
     _check_forward(base, inp, ref)
 
 
+def test_forward_run_to_run():
+    """Two calls on the same inputs: M is each slot's float32 updates applied in
+    time order by one stream, so its bits repeat; o sums each step's reads with
+    float reductions from many streams in no fixed order, so it may differ in
+    its last bits -- by float32 rounding of the sum, max |o1 - o2| / max |o| at
+    most 1e-6 (the parity bar against the oracle is 1e-4)."""
+    cfg = config(2).with_(B=1, H=4, T=1024)
+    d = to_device(gen_inputs(cfg, device="cuda"), cfg)
+    o1, M1 = gpu_forward(d, cfg)
+    o2, M2 = gpu_forward(d, cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(M1, M2)
+    spread = float((o1 - o2).abs().max() / o1.abs().max())
+    report("o run-to-run spread, pages-scale shape T=1024", [spread],
+           [float(((o1 - o2).abs() / (o1.abs() + 1e-6 * o1.abs().max())).max())])
+    assert spread <= 1e-6
+
+
 def test_fp32_wide_rows():
     cfg = config(0).with_(B=2, H=3, T=200, d_v=128, d_qk=24, n_sub=16, k=6, W=20, R=12,
                           m0_sd=1.0)
