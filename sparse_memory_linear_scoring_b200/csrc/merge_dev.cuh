@@ -43,6 +43,7 @@ __host__ __device__ inline MergeLayout merge_layout(const Plan& p, int warps) {
   L.Sk = p2(p.k);
   L.Sc = ((p.ncW > p.ncR ? p.ncW : p.ncR) + 31) & ~31;
   L.Ss = p2(p.W > p.R ? p.W : p.R);
+  if (L.Ss < 32) L.Ss = 32;  // the register sort of the selection takes 32 keys at least
   L.warps = warps;
   size_t o = 0;
   L.stair = o; o = al16(o + size_t(p.ncW + p.nfW + p.ncR + p.nfR + 2 * p.k) * 4);
@@ -136,6 +137,48 @@ __device__ __forceinline__ uint32_t warp_sort32_desc_u32(uint32_t x) {
     }
   }
   return x;
+}
+
+// Descending bitonic sort of 32 NJ 64-bit keys a[0..32 NJ) by one warp, in
+// registers: element j*32 + lane is lane's x[j]; partners 32 or more apart
+// are in the same lane, nearer ones are exchanged by shuffles.
+template <int NJ>
+__device__ inline void warp_sort_desc_reg(uint64_t* a) {
+  const int lane = threadIdx.x & 31;
+  constexpr int S = NJ * 32;
+  uint64_t x[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) x[j] = a[j * 32 + lane];
+#pragma unroll
+  for (int size = 2; size <= S; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {
+        const int js = stride / 32;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          if ((j & js) == 0) {
+            const bool desc = ((j * 32 + lane) & size) == 0;
+            const uint64_t lo = x[j], hi = x[j + js];
+            if (desc ? (lo < hi) : (lo > hi)) {
+              x[j] = hi;
+              x[j + js] = lo;
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const uint64_t y = __shfl_xor_sync(0xffffffffu, x[j], stride);
+          const bool desc = ((j * 32 + lane) & size) == 0;
+          const bool lower = (lane & stride) == 0;
+          x[j] = (lower == desc) ? (x[j] > y ? x[j] : y) : (x[j] < y ? x[j] : y);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) a[j * 32 + lane] = x[j];
 }
 
 // Ascending bitonic sort of S (power of two) 32-bit keys in shared memory by
@@ -406,10 +449,14 @@ __device__ inline void merge_one(const Plan& p, const uint2* sv1, int c1, const 
   }
   __syncwarp();
   if (sorted && !is_sorted) {
-    const int S = p2(n_sel);
+    const int S = p2(n_sel) < 32 ? 32 : p2(n_sel);
     for (int i = n_sel + lane; i < S; i += 32) sel[i] = 0;
     __syncwarp();
-    warp_sort_desc(sel, S);
+    if (S == 32) warp_sort_desc_reg<1>(sel);
+    else if (S == 64) warp_sort_desc_reg<2>(sel);
+    else if (S == 128) warp_sort_desc_reg<4>(sel);
+    else warp_sort_desc(sel, S);
+    __syncwarp();
   }
   // softmax over the selected float32 scores (the best candidate is (0, 0));
   // with sigmoid_w, the router weights of the selective-decay rule instead:
