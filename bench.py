@@ -747,6 +747,11 @@ def backward_bench(cfg, steps, warmup):
     bwd_ms = time_it(lambda: sdm.backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
                                           d["C1"], d["C2"], M0, *lists, d_o, dM, topk=cfg.k,
                                           workspace=ws))
+    # dL/dM_0 accumulated in dM_T's buffer (its values change from step to step,
+    # which does not change the work)
+    inpl_ms = time_it(lambda: sdm.backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                                           d["C1"], d["C2"], M0, *lists, d_o, dM, topk=cfg.k,
+                                           workspace=ws, dM_T_inplace=True))
     fwd_ms = time_it(lambda: sdm.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"],
                                          d["C2"], M, topk=cfg.k, W=cfg.W, R=cfg.R, o=o))
     clk = clocks.stop()
@@ -754,6 +759,7 @@ def backward_bench(cfg, steps, warmup):
     return {"backward": "sdm_backward at the forward's selections (gradients of q, k, v, "
                         "alpha, beta, C1, C2, M0)",
             "workload": workload_desc(cfg), "backward_ms": bwd_ms,
+            "backward_dM_in_place_ms": inpl_ms,
             "backward_token_heads_per_s": th / (bwd_ms / 1e3), "forward_ms": fwd_ms,
             "backward_over_forward_time": bwd_ms / fwd_ms, "workspace_bytes": ws.numel(),
             "steps": steps, "l2": "flushed before each step", "clocks": clk,

@@ -269,7 +269,9 @@ SDM_API const char* sdm_status_string(int status);
  * copied) and one byte per slot marking the rows written.
  * The codebook gradients are accumulated with float atomics, so their last
  * bits vary from call to call.  Same pointer, stream and error conventions as
- * sdm_forward (dalpha, dbeta: 4-byte alignment).
+ * sdm_forward (dalpha, dbeta: 4-byte alignment), with one exception to the
+ * no-alias rule: dM0 may be dM_T itself, and dL/dM_0 then accumulates in
+ * place (dM_T is overwritten), which saves copying it.
  */
 SDM_API size_t sdm_backward_workspace_bytes(const sdm_dims* dims);
 

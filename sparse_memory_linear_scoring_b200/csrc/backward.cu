@@ -380,7 +380,8 @@ extern "C" int sdm_backward(const void* q, const void* k, const void* v, const f
   float* Mw = reinterpret_cast<float*>(w + L.off_mw);
   uint8_t* touched = reinterpret_cast<uint8_t*>(w + L.off_touch);
   if (launch_init(p, st, s) != cudaSuccess) return SDM_ERR_CUDA;
-  // dM_0 = dM_T (or 0), dv = dC = 0, no row of the working table written yet
+  // dM_0 = dM_T (or 0; nothing to copy when dM0 is dM_T itself), dv = dC = 0,
+  // no row of the working table written yet
   if (cudaMemsetAsync(touched, 0, size_t(p.BH) * size_t(p.N), s) != cudaSuccess)
     return SDM_ERR_CUDA;
   {
@@ -388,7 +389,8 @@ extern "C" int sdm_backward(const void* q, const void* k, const void* v, const f
     const size_t nv4 = size_t(p.BH) * p.T * p.dv / 4;
     const size_t nc4 = size_t(p.H) * p.n * p.dh / 4;
     k_bwd_init<<<148 * 8, 256, 0, s>>>(
-        reinterpret_cast<const float4*>(dM_T), reinterpret_cast<float4*>(dM0), n4,
+        reinterpret_cast<const float4*>(dM_T), reinterpret_cast<float4*>(dM0),
+        static_cast<const void*>(dM_T) == static_cast<const void*>(dM0) ? 0 : n4,
         reinterpret_cast<float4*>(dv), nv4, reinterpret_cast<float4*>(dC1),
         reinterpret_cast<float4*>(dC2), p.dh % 4 == 0 ? nc4 : 0);
     if (cudaGetLastError() != cudaSuccess) return SDM_ERR_CUDA;

@@ -303,11 +303,13 @@ def step(q, k, v, alpha, beta, C1, C2, M, *, topk: int, W: int, R: int,
 
 
 def backward(q, k, v, alpha, beta, C1, C2, M0, idx_w, w_w, idx_r, w_r, d_o, dM_T=None, *,
-             topk: int, workspace: Optional[torch.Tensor] = None, stream=None):
+             topk: int, workspace: Optional[torch.Tensor] = None, stream=None,
+             dM_T_inplace: bool = False):
     """Gradients of the forward pass at its selections (sdm_backward).  M0 is the
     table the forward started from; the lists are sdm_select's; d_o = dL/do,
     dM_T = dL/dM_T (None: 0).  Returns a dict of float32 gradients: q, k, v,
-    alpha, beta, C1, C2, M0."""
+    alpha, beta, C1, C2, M0.  With dM_T_inplace, dL/dM_0 is accumulated in dM_T
+    itself (returned as "M0"), which saves copying it."""
     B, H, T, d_qk, n_sub, dt = _check_inputs(q, k, v, C1, C2, alpha, beta)
     d_v = v.shape[-1]
     W, R = idx_w.shape[-1], idx_r.shape[-1]
@@ -327,7 +329,10 @@ def backward(q, k, v, alpha, beta, C1, C2, M0, idx_w, w_w, idx_r, w_r, d_o, dM_T
     g = dict(q=torch.empty(B, H, T, d_qk, **f32), k=torch.empty(B, H, T, d_qk, **f32),
              v=torch.empty(B, H, T, d_v, **f32), alpha=torch.empty(B, H, T, **f32),
              beta=torch.empty(B, H, T, **f32), C1=torch.empty(H, n_sub, d_qk // 2, **f32),
-             C2=torch.empty(H, n_sub, d_qk // 2, **f32), M0=torch.empty(B, H, N, d_v, **f32))
+             C2=torch.empty(H, n_sub, d_qk // 2, **f32),
+             M0=dM_T if (dM_T_inplace and dM_T is not None) else torch.empty(B, H, N, d_v, **f32))
+    if dM_T_inplace and (dM_T is None or not dM_T.is_contiguous()):
+        raise ValueError("dM_T_inplace needs a contiguous dM_T")
     lib = load_library()
     need = int(lib.sdm_backward_workspace_bytes(ctypes.byref(dims)))
     if need == 0:

@@ -54,3 +54,31 @@ def test_backward_against_reference(cfg):
             used[np.unique(ref_fwd["idx_w"][b, h])] = True
             used[np.unique(ref_fwd["idx_r"][b, h])] = True
             assert np.array_equal(gM[b, h][~used], dM[b, h][~used])
+
+
+def test_backward_dM_in_place():
+    """dM0 given as dM_T itself: the same gradients, with dM_T overwritten by
+    dL/dM_0 -- bit for bit where each value has one writer (dM_0: each slot's g
+    is carried by one stream; dq, dk, dalpha, dbeta), to float rounding where
+    float reductions from many streams add up (dv, dC1, dC2)."""
+    cfg = config(1).with_(B=1, H=2, T=100, n_sub=64, k=16, W=32, R=32, d_v=16, m0_sd=0.5)
+    inp = gen_inputs(cfg)
+    d = to_device(inp, cfg)
+    lists = sdm.select(d["q"], d["k"], d["C1"], d["C2"], topk=cfg.k, W=cfg.W, R=cfg.R,
+                       d_v=cfg.d_v)
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    do = torch.randn(cfg.B, cfg.H, cfg.T, cfg.d_v, device="cuda", generator=gen)
+    dM = torch.randn(cfg.B, cfg.H, cfg.N, cfg.d_v, device="cuda", generator=gen)
+    args = (d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["C1"], d["C2"], d["M"], *lists, do)
+    g1 = sdm.backward(*args, dM, topk=cfg.k)
+    dM2 = dM.clone()
+    g2 = sdm.backward(*args, dM2, topk=cfg.k, dM_T_inplace=True)
+    torch.cuda.synchronize()
+    assert g2["M0"].data_ptr() == dM2.data_ptr()
+    assert torch.equal(g1["M0"], dM2)
+    for name in ("q", "k", "alpha", "beta"):
+        assert torch.equal(g1[name], g2[name]), name
+    for name in ("v", "C1", "C2"):
+        a, b = g1[name], g2[name]
+        assert float((a - b).abs().max()) <= 1e-5 * float(a.abs().max()), name
+
