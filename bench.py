@@ -520,7 +520,8 @@ def run_reference(args, cfg):
     value = th / tot
     sample = "%d heads x first %d steps of %s per step (oracle C, float64, %d threads)" % (
         nheads, T_s, cfg.name, min(nthr, nheads))
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workload_desc(cfg), "sample": sample},
